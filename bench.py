@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Benchmark of the bifocal attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline (``value``): bifocal prefill TFLOP/s at L = 131072 with Qwen3-8B attention heads
+(Hq 32, Hkv 8, D 128), w_pretrained 32768 (G = 4), w0 4096, frequency interpolation,
+counted as 2 * 2 * (L^2 / 2) * D * Hq FLOP per prefill. One step = one full prefill
+(RoPE pass + fused attention) over inputs already resident in HBM (1.5 GB, larger than
+L2). The same run also times: the attention kernel alone (roofline), the plain causal
+RoPE comparator (overhead), the 200-step decode across the G = 4 -> 5 change (us/step and
+GB/s vs HBM), the end-to-end call with host buffers, and the fp64 CPU oracle on a bounded
+sample of the same workload (cpu_baseline). Multi-GPU runs are replicas (weak scaling):
+each rank runs the same workload; value = all ranks' FLOPs / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "bifocal prefill TFLOP/s at 128K (frac of BF16 peak); decode µs/step vs HBM"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------ distributed plumbing
+class Dist:
+    def __init__(self, want_pg: bool):
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+        if want_pg and self.world > 1:
+            import datetime
+
+            import torch
+            import torch.distributed as dist
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch
+        import torch.distributed as dist
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ clocks sampler
+class Clocks:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            cmd += ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            pass
+        self.cmd = cmd
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ timing helpers
+def time_loop(fn, steps, warmup, dist, torch):
+    """Device time of `steps` calls of fn (CUDA events on the current stream), max over ranks."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    return dist.max(s.elapsed_time(e))
+
+
+def cpu_info():
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:
+        cores = os.cpu_count() or 1
+    threads = cores
+    try:
+        from threadpoolctl import threadpool_info
+        ti = [x for x in threadpool_info() if x.get("user_api") == "blas"]
+        if ti:
+            threads = int(ti[0].get("num_threads", cores))
+    except Exception:
+        pass
+    return cores, threads
+
+
+def oracle_sample(q, k, v, w, rows, heads):
+    """Time the fp64 oracle on (rows x heads) of the prefill workload; returns (seconds, counted FLOPs)."""
+    import numpy as np
+
+    import oracle.bifocal_ref as R
+    g = w.hq // w.hkv
+    t0 = time.perf_counter()
+    for h in heads:
+        qh = q[:, :, h:h + 1].float().double().numpy()
+        kh = k[:, :, h // g:h // g + 1].float().double().numpy()
+        vh = v[:, :, h // g:h // g + 1].float().double().numpy()
+        R.bifocal_attention(qh, kh, vh, w.w0, w.w_pretrained, w.theta, w.mode, rows=np.asarray(rows))
+    dt = time.perf_counter() - t0
+    flops = sum(4.0 * w.head_dim * (r + 1) for r in rows) * len(heads)
+    return dt, flops
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    """The fp64 CPU oracle as the reference arm, on bounded samples of the same workload."""
+    import seeded_inputs as si
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = si.qwen3_8b_128k(args.w0)
+    q, k, v = si.prefill_inputs(w)
+    rows = [w.L - 1]
+    heads = list(range(8))
+    times, flops = [], 0.0
+    for i in range(args.warmup + args.steps):
+        dt, fl = oracle_sample(q, k, v, w, rows, heads)
+        if i >= args.warmup:
+            times.append(dt)
+            flops = fl
+    ms = 1000.0 * statistics.mean(times)
+    value = flops / (ms / 1000.0) / 1e12
+    cores, threads = cpu_info()
+    sample = f"query row {rows[0]} of query heads 0-7 per step (fp64 NumPy oracle, both RoPE branches over all keys)"
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    G = max(1, -(-w.L // w.w_pretrained))  # for the record only; the library computes its own
+    return {"workload": w.name, "batch": 1, "L": w.L, "hq": w.hq, "hkv": w.hkv, "head_dim": w.head_dim, "w0": w.w0,
+            "w_pretrained": w.w_pretrained, "G": G, "mode": w.mode, "theta": w.theta, "seed": w.seed,
+            "l2": "inputs larger than L2 (q+k+v 1.5 GB bf16)", "parallelism": "replicas"}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+
+    import rope_context_extension_bifocal_b200 as bfl
+    import seeded_inputs as si
+
+    dist = Dist(want_pg=True)
+    torch.cuda.set_device(dist.local)
+    dev = torch.device("cuda", dist.local)
+    peaks, peak_kind = load_peaks()
+    launches = 0
+
+    w = si.qwen3_8b_128k(args.w0)
+    q_h, k_h, v_h = si.prefill_inputs(w)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    params = bfl.make_params(w.hq, w.hkv, w.head_dim, w.w0, w.w_pretrained, w.theta, w.mode)
+    ws = torch.empty(bfl.prefill_workspace_size(bfl.DTYPE_BF16, 1, w.L, params), dtype=torch.uint8, device=dev)
+    out = torch.empty(1, w.L, w.hq, w.head_dim, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(1, w.hq, w.L, dtype=torch.float32, device=dev)
+    flops = w.causal_flops
+
+    def step_rope():
+        bfl.bifocal_prefill_rope(q, k, v, params, ws)
+
+    def step_attn():
+        bfl.bifocal_prefill_attention(v, params, ws, out, lse)
+
+    # ---- headline: K full prefills, per-kernel events inside the timed region
+    for _ in range(args.warmup):
+        step_rope()
+        step_attn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = Clocks(dist.local)
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        ev[i][0].record()
+        step_rope()
+        ev[i][1].record()
+        step_attn()
+        ev[i][2].record()
+        launches += 2
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dist.barrier()
+    total_ms = dist.max(ev[0][0].elapsed_time(ev[-1][2]))
+    attn_ms = dist.max(statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
+    rope_ms = dist.max(statistics.mean(e[0].elapsed_time(e[1]) for e in ev))
+    ms_per_step = total_ms / args.steps
+    value = flops * dist.world / (ms_per_step / 1e3) / 1e12
+    attn_tflops = flops / (attn_ms / 1e3) / 1e12
+    peak_t = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    roofline = {"bound": "tensor", "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                "frac": attn_tflops / peak_t, "traffic": None, "kernel": "bifocal attention (prefill)",
+                "peak_kind": f"{peak_kind} bf16 dense burst", "kernel_ms": attn_ms, "rope_pass_ms": rope_ms}
+
+    # ---- plain comparator (same shapes, original RoPE only)
+    def step_plain():
+        bfl.rope_causal_prefill(q, k, v, theta=w.theta, out=out, workspace=ws)
+
+    plain_ms = time_loop(step_plain, max(2, args.steps // 2), 1, dist, torch) / max(2, args.steps // 2)
+    overhead_prefill = ms_per_step / plain_ms - 1.0
+
+    # ---- w0 sweep of the 128K config (short)
+    sweep = {}
+    if not args.no_sweep:
+        for w0 in si.QWEN3_8B_128K_W0:
+            p2 = bfl.make_params(w.hq, w.hkv, w.head_dim, w0, w.w_pretrained, w.theta, w.mode)
+
+            def step_sweep(p2=p2):
+                bfl.bifocal_prefill_rope(q, k, v, p2, ws)
+                bfl.bifocal_prefill_attention(v, p2, ws, out, lse)
+
+            ms = time_loop(step_sweep, 2, 1, dist, torch) / 2
+            sweep[str(w0)] = {"ms": ms, "tflops": flops / (ms / 1e3) / 1e12}
+
+    # ---- end to end through the public call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+        def step_e2e():
+            q.copy_(qp, non_blocking=True)
+            k.copy_(kp, non_blocking=True)
+            v.copy_(vp, non_blocking=True)
+            bfl.bifocal_prefill(q, k, v, w0=w.w0, w_pretrained=w.w_pretrained, theta=w.theta, mode=w.mode, out=out,
+                                workspace=ws)
+            out_h.copy_(out, non_blocking=True)
+            lse_h.copy_(lse, non_blocking=True)
+
+        n_e2e = max(2, args.steps // 2)
+        e2e_ms = time_loop(step_e2e, n_e2e, 1, dist, torch) / n_e2e
+        h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+        d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+        e2e = {"value": flops * dist.world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        del qp, kp, vp, out_h, lse_h
+
+    # ---- decode: 200 steps across the G = 4 -> 5 change
+    decode = None
+    if not args.no_decode:
+        del ws
+        torch.cuda.empty_cache()
+        decode = run_decode(args, torch, bfl, si, dev, peaks, peak_kind)
+
+    # ---- CPU baseline: the oracle on a bounded sample, rank 0, N = 1 only
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        rows = list(range(w.L - 8, w.L))
+        dt, fl = oracle_sample(q_h, k_h, v_h, w, rows, list(range(w.hq)))
+        cores, threads = cpu_info()
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"query rows {rows[0]}-{rows[-1]} x all {w.hq} heads of the same workload "
+                         f"(fp64 NumPy, {dt:.1f} s; host has {cores} usable cores)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": dist.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "precision": {"inputs": "bf16", "qk_operands": "f16", "pv_operands": "bf16", "accumulate": "f32"},
+        "data": "synthetic: q/k/v iid N(0,1) bf16, torch CPU generator seed 3 (Qwen3-8B attention shapes)",
+        "config": workload_config(w),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clk,
+        "gpu_launches": launches,
+        "overhead_vs_plain": {"prefill": overhead_prefill, "prefill_plain_ms": plain_ms,
+                              "decode": decode["overhead_vs_plain"] if decode else None},
+        "w0_sweep": sweep,
+        "decode": decode,
+        "build": bfl.build_info(),
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+def run_decode(args, torch, bfl, si, dev, peaks, peak_kind):
+    w = si.DECODE_128K
+    stream = si.DecodeStream(w)
+    kp, vp = stream.cache_prefix()
+    kcache = torch.zeros(w.capacity, w.hkv, w.head_dim, dtype=torch.bfloat16, device=dev)
+    vcache = torch.zeros_like(kcache)
+    kcache[:w.prefix_len] = kp.to(dev)
+    vcache[:w.prefix_len] = vp.to(dev)
+    del kp, vp
+    steps = [tuple(t.to(dev) for t in stream.step()) for _ in range(args.decode_steps)]
+    params = bfl.make_params(w.hq, w.hkv, w.head_dim, w.w0, w.w_pretrained, w.theta, w.mode)
+    ws = torch.empty(bfl.decode_workspace_size(w.capacity, params), dtype=torch.uint8, device=dev)
+    out = torch.empty(w.hq, w.head_dim, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(w.hq, dtype=torch.float32, device=dev)
+
+    def session(fn):
+        for t in range(min(args.warmup, len(steps))):  # warm-up rewrites the same rows the session writes
+            fn(t)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in steps]
+        for t in range(len(steps)):
+            ev[t][0].record()
+            fn(t)
+            ev[t][1].record()
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) * 1e3 for a, b in ev]  # us
+
+    def bif(t):
+        q, kn, vn = steps[t]
+        bfl.bifocal_decode(q, kn, vn, kcache, vcache, w.prefix_len + t + 1, w0=w.w0, w_pretrained=w.w_pretrained,
+                           theta=w.theta, mode=w.mode, out=out, workspace=ws)
+
+    def plain(t):
+        q, kn, vn = steps[t]
+        bfl.rope_causal_decode(q, kn, vn, kcache, vcache, w.prefix_len + t + 1, theta=w.theta, out=out,
+                               workspace=ws)
+
+    us = session(bif)
+    us_plain = session(plain)
+    gbs = [w.cache_bytes(w.prefix_len + t + 1) / (u * 1e-6) / 1e9 for t, u in enumerate(us)]
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    med = statistics.median(us)
+    med_gbs = statistics.median(gbs)
+    srt = sorted(us)
+    return {
+        "workload": w.name, "steps": len(us), "us_mean": statistics.mean(us), "us_median": med,
+        "us_p95": srt[min(len(srt) - 1, int(0.95 * len(srt)))], "us_min": srt[0],
+        "gbs_median": med_gbs, "us_steps_70_75": us[70:76], "G_steps_70_75": [
+            bfl.bifocal_factor(w.prefix_len + t + 1, w.w_pretrained) for t in range(70, 76)],
+        "overhead_vs_plain": statistics.median(us) / statistics.median(us_plain) - 1.0,
+        "plain_us_median": statistics.median(us_plain),
+        "roofline": {"bound": "hbm", "achieved": med_gbs, "peak": hbm, "unit": "GB/s", "frac": med_gbs / hbm,
+                     "traffic": None, "kernel": "decode step (append + split-KV partial + combine)",
+                     "peak_kind": f"{peak_kind} HBM copy",
+                     "bytes_per_step_at_131072": w.cache_bytes(131072)},
+        "gpu_launches": 3 * len(us),
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--w0", type=int, default=4096)
+    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,175 @@
+/*
+ * bifocal.h - C ABI of the B200 (sm_100a) Dynamic Bifocal RoPE attention library.
+ *
+ * Method: Jet-Long, "Efficient Long-Context Extension with Dynamic Bifocal RoPE"
+ * (arXiv 2607.07740), as described by
+ *   [VS] the video script "Tom 视频脚本镜像 · arXiv 2607.07740 · Jet-Long"
+ *        (section 3 voice-over; section 4 storyboard, scene-2 formula),
+ *   [AF] the ai-feeds summary "Jet-Long: 使用动态双焦点RoPE的高效长上下文扩展"
+ *        (section 方法: input statement, key modules 1-4, output statement;
+ *         section 实验: key findings / ablation),
+ *   [KB] the knowledge-base note "Jet-Long：动态双焦点 RoPE 长上下文扩展" (设计原理),
+ *   [SN] the seventnews article "L'attention bifocale de Jet-Long tue le compromis
+ *        de mise à l'échelle fixe pour les LLM à long contexte".
+ *
+ * What every attention entry point computes, per query row i and key j <= i
+ * (0-based positions, rotate-half RoPE pairing k <-> k + D/2, omega_k = theta^(-2k/D)):
+ *   score(i, j) = scale * < R_orig(i) q_i , R_orig(j) k_j >   if i - j <  w0   (local window, [AF] module 1)
+ *               = scale * < R_long(i) q_i , R_long(j) k_j >   if i - j >= w0   (long range,   [AF] module 1)
+ *   R_orig(p) rotates pair k by p * omega_k. R_long(p) rotates pair k by
+ *     p * omega_k / G          (BF_MODE_FREQ_INTERP, frequency interpolation), or
+ *     floor(p / G) * omega_k   (BF_MODE_POS_ALIAS, position aliasing);
+ *   both named by the ablation in [AF] 实验.  G = max(1, ceil(L / w_pretrained)) ([VS] scene-2).
+ *   out_i = softmax_j(score(i, .)) . v ;  lse_i = m_i + ln(sum_j exp(score(i,j) - m_i)).
+ * This equals the inclusion-exclusion merge of [AF] module 3 / [SN] (long branch over all keys,
+ * minus the long branch on the band, plus the local branch on the band, in log-sum-exp form);
+ * the kernels evaluate it as one online softmax that picks the branch per (i, j).
+ *
+ * Conventions shared by all calls
+ *   - Tensor pointers are DEVICE pointers on the current CUDA device, contiguous,
+ *     row-major, and owned by the caller. The library never allocates device memory
+ *     on a call path: scratch space is a caller-provided workspace whose size the
+ *     matching *_workspace_size call returns (256-byte aligned pointer required).
+ *   - q and k are RAW (pre-RoPE). RoPE and the correction rotation are applied by the
+ *     library. The KV cache holds keys under the ORIGINAL RoPE, in bf16.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Errors: argument errors return BF_ERR_INVALID / BF_ERR_UNSUPPORTED / BF_ERR_WORKSPACE
+ *     before any launch; a failed launch returns BF_ERR_CUDA. No call traps, aborts or prints.
+ *     Device-side bounded waits that expire set a device status word, read (and cleared)
+ *     by bifocal_last_device_error().
+ */
+#ifndef BIFOCAL_H_
+#define BIFOCAL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BF_API __attribute__((visibility("default")))
+#else
+#define BF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BF_OK = 0,
+  BF_ERR_INVALID = 1,      /* bad pointer, size, shape or parameter */
+  BF_ERR_UNSUPPORTED = 2,  /* valid but not built: head_dim not in {64, 128}, unknown dtype */
+  BF_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  BF_ERR_TIMEOUT = 4,      /* a device-side bounded wait expired (reported by bifocal_last_device_error) */
+  BF_ERR_WORKSPACE = 5,    /* workspace missing, misaligned or smaller than *_workspace_size */
+  BF_ERR_NO_DEVICE = 6     /* no CUDA device, or the device is not sm_100 */
+} bf_status_t;
+
+typedef enum { BF_MODE_FREQ_INTERP = 0, BF_MODE_POS_ALIAS = 1 } bf_mode_t;
+typedef enum { BF_DTYPE_BF16 = 0, BF_DTYPE_FP32 = 1 } bf_dtype_t;
+
+/* flags */
+#define BF_FLAG_FORCE_BIFOCAL 1 /* run the two-branch kernel even when G == 1 or w0 >= L (results are equal) */
+
+typedef struct {
+  int32_t hq;           /* query heads; hq % hkv == 0; query head h reads kv head h / (hq / hkv) */
+  int32_t hkv;          /* key/value heads */
+  int32_t head_dim;     /* D: 64 or 128 */
+  int32_t w0;           /* local window: pairs with i - j < w0 use the original RoPE; w0 >= 0 */
+  int32_t w_pretrained; /* pretrained context window, >= 1; sets G */
+  int32_t mode;         /* bf_mode_t */
+  double rope_theta;    /* RoPE base theta > 1 */
+  float softmax_scale;  /* 0 => 1/sqrt(head_dim) */
+  int32_t flags;        /* BF_FLAG_* */
+} bf_params_t;
+
+/* Dynamic factor G = max(1, ceil(L / w_pretrained)) ([VS] storyboard scene-2; [AF] module 2).
+ * Host only, no CUDA call. Returns -1 when L < 0 or w_pretrained < 1. */
+BF_API int32_t bifocal_factor(int64_t L, int32_t w_pretrained);
+
+/* Bytes of device workspace bifocal_prefill / rope_causal_prefill need for these sizes and
+ * this input dtype: the rotated query and key forms (bf16) and, for fp32 inputs, a bf16
+ * copy of v. Host only. Returns 0 on invalid arguments. */
+BF_API size_t bifocal_prefill_workspace_size(int32_t dtype, int32_t batch, int32_t L, const bf_params_t* p);
+
+/* Bifocal causal prefill ([AF] 方法: input = sequence length L and the pretrained RoPE
+ * configuration; output = the attention output of the current sequence).
+ *   q    [batch, L, hq,  D]  raw, dtype (bf16 or fp32)
+ *   k, v [batch, L, hkv, D]  raw, dtype
+ *   out  [batch, L, hq,  D]  bf16, written
+ *   lse  [batch, hq, L]      fp32 natural-log LSE of the scaled scores, written (may be NULL)
+ *   kcache_out [batch, L, hkv, D] bf16: keys under the original RoPE (the decode cache); may be NULL
+ *   vcache_out [batch, L, hkv, D] bf16: copy of v in bf16; may be NULL
+ *   workspace / ws_bytes: >= bifocal_prefill_workspace_size(dtype, batch, L, p), 256-byte aligned.
+ * G is taken once from L. When G == 1 or w0 >= L every pair is local and the call runs the
+ * plain kernel (identical result) unless BF_FLAG_FORCE_BIFOCAL is set.
+ * Errors: BF_ERR_INVALID for NULL q/k/v/out/p, L < 1, batch < 1, hq % hkv != 0, w0 < 0,
+ * w_pretrained < 1, theta <= 1, unknown mode; BF_ERR_UNSUPPORTED for head_dim not 64/128 or
+ * an unknown dtype; BF_ERR_WORKSPACE for a short/misaligned workspace; BF_ERR_CUDA on launch failure. */
+BF_API bf_status_t bifocal_prefill(const void* q, const void* k, const void* v, int32_t dtype, int32_t batch, int32_t L,
+                            const bf_params_t* p, void* out, float* lse, void* kcache_out, void* vcache_out,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/* The two steps of bifocal_prefill, for callers that schedule or time them apart.
+ * Step 1 (RoPE pass): one HBM pass over the raw q and k that writes, into the workspace, the
+ *   QK^T operands under the original and the long-range RoPE (fp16, head-major), a bf16 copy
+ *   of fp32 v, and kcache_out / vcache_out when given.
+ * Step 2 (attention): the fused two-branch causal attention over those operands and v
+ *   (v as passed to step 1), writing out and lse.
+ * Both take the arguments of bifocal_prefill; step 2 must see the same q/k/v dtype, batch, L,
+ * p and workspace as the step 1 that precedes it on the stream. Errors as bifocal_prefill. */
+BF_API bf_status_t bifocal_prefill_rope(const void* q, const void* k, const void* v, int32_t dtype, int32_t batch,
+                                        int32_t L, const bf_params_t* p, void* kcache_out, void* vcache_out,
+                                        void* workspace, size_t ws_bytes, void* stream);
+BF_API bf_status_t bifocal_prefill_attention(const void* v, int32_t dtype, int32_t batch, int32_t L,
+                                             const bf_params_t* p, void* out, float* lse, void* workspace,
+                                             size_t ws_bytes, void* stream);
+
+/* Plain causal attention under the original RoPE: the same kernels with the long branch
+ * compiled out (the comparator for the bifocal overhead). Same arguments as bifocal_prefill;
+ * w0, w_pretrained and mode are ignored. */
+BF_API bf_status_t rope_causal_prefill(const void* q, const void* k, const void* v, int32_t dtype, int32_t batch, int32_t L,
+                                const bf_params_t* p, void* out, float* lse, void* kcache_out, void* vcache_out,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace bifocal_decode / rope_causal_decode need for a cache of up to
+ * L_max rows: the split-KV partial results (fp32). Host only. 0 on invalid arguments. */
+BF_API size_t bifocal_decode_workspace_size(int32_t L_max, const bf_params_t* p);
+
+/* One single-batch decode step ([AF] module 3: on-the-fly correction rotation of cached keys;
+ * [KB] 设计原理: the near/far boundary slides as tokens are generated).
+ *   q      [hq,  D] bf16 raw query of the new token, at position p = L - 1
+ *   k_new  [hkv, D] bf16 raw key of the new token;  v_new [hkv, D] bf16
+ *   kcache [cap, hkv, D] bf16 keys under the ORIGINAL RoPE; rows 0..L-2 valid on entry.
+ *          Row L-1 is written with R_orig(L-1) k_new (the append step).
+ *   vcache [cap, hkv, D] bf16; row L-1 is written with v_new.
+ *   L      length including the new token, 1 <= L <= cap. G = max(1, ceil(L / w_pretrained)).
+ *   out    [hq, D] bf16;  lse [hq] fp32 (may be NULL).
+ *   workspace / ws_bytes: >= bifocal_decode_workspace_size(L, p), 256-byte aligned.
+ * Cached key j takes part in the long branch through the correction rotation
+ * R_long(j) R_orig(j)^-1, applied in registers while it streams from HBM; the cache itself
+ * is never rewritten and no second key copy exists.
+ * Errors: as bifocal_prefill; BF_ERR_INVALID also for L > cap. */
+BF_API bf_status_t bifocal_decode(const void* q, const void* k_new, const void* v_new, void* kcache, void* vcache,
+                           int32_t cap, int32_t L, const bf_params_t* p, void* out, float* lse, void* workspace,
+                           size_t ws_bytes, void* stream);
+
+/* Plain-RoPE decode step (comparator): same arguments; every cached key is used as stored. */
+BF_API bf_status_t rope_causal_decode(const void* q, const void* k_new, const void* v_new, void* kcache, void* vcache,
+                               int32_t cap, int32_t L, const bf_params_t* p, void* out, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+BF_API const char* bifocal_status_string(int32_t status);
+
+/* Reads and clears the device status word that bounded waits set when they expire on the
+ * current device. Synchronises `stream` first. Returns BF_OK, BF_ERR_TIMEOUT or BF_ERR_CUDA. */
+BF_API bf_status_t bifocal_last_device_error(void* stream);
+
+/* Library build identification (static string): kernels compiled in and their target. */
+BF_API const char* bifocal_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BIFOCAL_H_ */

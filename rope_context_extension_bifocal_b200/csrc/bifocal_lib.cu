@@ -1,0 +1,441 @@
+// C-ABI library: argument validation, dynamic factor, workspace layout, TMA
+// descriptors and kernel dispatch. Built as one translation unit with the kernels so
+// that the device status word is a single object.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/bifocal.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill_mma.cuh"
+#include "rope_prepass.cuh"
+
+namespace {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int kMaxSplits = 320;  // split-KV partials reserved in the decode workspace
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct Rope {
+  double omega[64];
+  double omega_long[64];
+  double omega_corr[64];
+};
+
+// omega_k = theta^(-2k/D) in fp64 on the host; long-range forms for factor G.
+Rope make_rope(double theta, int D, int G) {
+  Rope r;
+  std::memset(&r, 0, sizeof(r));
+  for (int k = 0; k < D / 2; ++k) {
+    const double om = std::pow(theta, -2.0 * k / D);
+    r.omega[k] = om;
+    r.omega_long[k] = om / G;
+    r.omega_corr[k] = om / G - om;
+  }
+  return r;
+}
+
+int factor(int64_t L, int w) { return L <= w ? 1 : static_cast<int>((L + w - 1) / w); }
+
+bf_status_t check_params(const bf_params_t* p, bool need_window) {
+  if (!p) return BF_ERR_INVALID;
+  if (p->hq < 1 || p->hkv < 1 || p->hq % p->hkv) return BF_ERR_INVALID;
+  if (p->head_dim != 64 && p->head_dim != 128) return BF_ERR_UNSUPPORTED;
+  if (!(p->rope_theta > 1.0) || !std::isfinite(p->rope_theta)) return BF_ERR_INVALID;
+  if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale)) return BF_ERR_INVALID;
+  if (need_window) {
+    if (p->w0 < 0 || p->w_pretrained < 1) return BF_ERR_INVALID;
+    if (p->mode != BF_MODE_FREQ_INTERP && p->mode != BF_MODE_POS_ALIAS) return BF_ERR_INVALID;
+  }
+  return BF_OK;
+}
+
+float scale_log2(const bf_params_t* p) {
+  const double s = p->softmax_scale > 0.f ? p->softmax_scale : 1.0 / std::sqrt(static_cast<double>(p->head_dim));
+  return static_cast<float>(s * 1.4426950408889634073599246810019);
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// Cache [cap, hkv, D] bf16 viewed as (d_lo = 64, d_hi = D/64, head, key) with a box of
+// (64, 1, 1, kb) and the 128-byte swizzle: one 128-byte row per key.
+bool make_cache_map(CUtensorMap* map, const void* base, int cap, int hkv, int D, int kb) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(D / 64), static_cast<cuuint64_t>(hkv), static_cast<cuuint64_t>(cap)};
+  cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(hkv) * D * 2};
+  cuuint32_t box[4] = {64, 1, 1, static_cast<cuuint32_t>(kb)};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ------------------------------------------------------------------ prefill
+struct PrefillLayout {
+  size_t qo, ql, ko, kl, vb, total;
+};
+
+PrefillLayout prefill_layout(int dtype, int batch, int L, const bf_params_t* p) {
+  PrefillLayout w{};
+  const size_t qbytes = align256(static_cast<size_t>(batch) * L * p->hq * p->head_dim * 2);
+  const size_t kbytes = align256(static_cast<size_t>(batch) * L * p->hkv * p->head_dim * 2);
+  w.qo = 0;
+  w.ql = w.qo + qbytes;
+  w.ko = w.ql + qbytes;
+  w.kl = w.ko + kbytes;
+  w.vb = w.kl + kbytes;
+  w.total = w.vb + (dtype == BF_DTYPE_FP32 ? kbytes : 0);
+  return w;
+}
+
+template <int D, bool BIF>
+cudaError_t launch_attn_mma(const bf::AttnArgs& a, int batch, cudaStream_t st) {
+  constexpr int smem = bf::attn_mma_smem_bytes<D, BIF>();
+  cudaError_t e = cudaFuncSetAttribute(bf::attn_mma_kernel<D, BIF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.L + bf::mma_cfg::BM - 1) / bf::mma_cfg::BM, a.hq, batch);
+  bf::attn_mma_kernel<D, BIF><<<grid, bf::mma_cfg::WARPS * 32, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+// What a prefill call resolves before any launch (shared by the one-call form and the
+// two steps, so both make the same choice).
+struct PrefillPlan {
+  int D, G;
+  bool bif;  // two-branch kernel (else every pair is local: the plain kernel gives the same result)
+  PrefillLayout lay;
+  Rope rope;
+};
+
+bf_status_t plan_prefill(bool bifocal_api, int32_t dtype, int32_t batch, int32_t L, const bf_params_t* p,
+                         void* workspace, size_t ws_bytes, PrefillPlan* plan) {
+  bf_status_t s = check_params(p, bifocal_api);
+  if (s != BF_OK) return s;
+  if (batch < 1 || L < 1) return BF_ERR_INVALID;
+  if (dtype != BF_DTYPE_BF16 && dtype != BF_DTYPE_FP32) return BF_ERR_UNSUPPORTED;
+  plan->lay = prefill_layout(dtype, batch, L, p);
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < plan->lay.total) return BF_ERR_WORKSPACE;
+  plan->D = p->head_dim;
+  plan->G = bifocal_api ? factor(L, p->w_pretrained) : 1;
+  plan->bif = bifocal_api && ((p->flags & BF_FLAG_FORCE_BIFOCAL) || (plan->G > 1 && p->w0 < L));
+  plan->rope = make_rope(p->rope_theta, plan->D, plan->G);
+  return BF_OK;
+}
+
+bf_status_t prefill_rope_impl(bool bifocal_api, const void* q, const void* k, const void* v, int32_t dtype,
+                              int32_t batch, int32_t L, const bf_params_t* p, void* kcache_out, void* vcache_out,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  PrefillPlan plan;
+  bf_status_t s = check_params(p, bifocal_api);
+  if (s != BF_OK) return s;
+  if (!q || !k || !v) return BF_ERR_INVALID;
+  const size_t align_in = dtype == BF_DTYPE_FP32 ? 32 : 16;
+  if (!aligned(q, align_in) || !aligned(k, align_in) || !aligned(v, align_in)) return BF_ERR_INVALID;
+  if ((kcache_out && !aligned(kcache_out, 16)) || (vcache_out && !aligned(vcache_out, 16))) return BF_ERR_INVALID;
+  s = plan_prefill(bifocal_api, dtype, batch, L, p, workspace, ws_bytes, &plan);
+  if (s != BF_OK) return s;
+  const int D = plan.D;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  bf::PrepassArgs pa{};
+  pa.q = q;
+  pa.k = k;
+  pa.v = v;
+  pa.batch = batch;
+  pa.L = L;
+  pa.hq = p->hq;
+  pa.hkv = p->hkv;
+  pa.G = plan.G;
+  pa.mode = bifocal_api ? p->mode : 0;
+  pa.need_long = plan.bif ? 1 : 0;
+  pa.Qo = reinterpret_cast<__half*>(ws + plan.lay.qo);
+  pa.Ql = reinterpret_cast<__half*>(ws + plan.lay.ql);
+  pa.Ko = reinterpret_cast<__half*>(ws + plan.lay.ko);
+  pa.Kl = reinterpret_cast<__half*>(ws + plan.lay.kl);
+  pa.Vb = dtype == BF_DTYPE_FP32 ? reinterpret_cast<bf16*>(ws + plan.lay.vb) : nullptr;
+  pa.kcache = static_cast<bf16*>(kcache_out);
+  pa.vcache = static_cast<bf16*>(vcache_out);
+  std::memcpy(pa.omega, plan.rope.omega, sizeof(pa.omega));
+  std::memcpy(pa.omega_long, plan.rope.omega_long, sizeof(pa.omega_long));
+  const long long rows = static_cast<long long>(batch) * L;
+  const dim3 pgrid(static_cast<unsigned>((rows + 7) / 8));
+  if (dtype == BF_DTYPE_BF16) {
+    if (D == 128)
+      bf::rope_prepass_kernel<bf16, 128><<<pgrid, 256, 0, st>>>(pa);
+    else
+      bf::rope_prepass_kernel<bf16, 64><<<pgrid, 256, 0, st>>>(pa);
+  } else {
+    if (D == 128)
+      bf::rope_prepass_kernel<float, 128><<<pgrid, 256, 0, st>>>(pa);
+    else
+      bf::rope_prepass_kernel<float, 64><<<pgrid, 256, 0, st>>>(pa);
+  }
+  return cudaGetLastError() == cudaSuccess ? BF_OK : BF_ERR_CUDA;
+}
+
+bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtype, int32_t batch, int32_t L,
+                                   const bf_params_t* p, void* out, float* lse, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+  PrefillPlan plan;
+  bf_status_t s = check_params(p, bifocal_api);
+  if (s != BF_OK) return s;
+  if (!v || !out) return BF_ERR_INVALID;
+  if (!aligned(v, dtype == BF_DTYPE_FP32 ? 32 : 16) || !aligned(out, 16) || (lse && !aligned(lse, 4)))
+    return BF_ERR_INVALID;
+  s = plan_prefill(bifocal_api, dtype, batch, L, p, workspace, ws_bytes, &plan);
+  if (s != BF_OK) return s;
+  const int D = plan.D;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  bf::AttnArgs aa{};
+  aa.Qo = reinterpret_cast<const __half*>(ws + plan.lay.qo);
+  aa.Ql = reinterpret_cast<const __half*>(ws + plan.lay.ql);
+  aa.Ko = reinterpret_cast<const __half*>(ws + plan.lay.ko);
+  aa.Kl = reinterpret_cast<const __half*>(ws + plan.lay.kl);
+  aa.V = dtype == BF_DTYPE_FP32 ? reinterpret_cast<const bf16*>(ws + plan.lay.vb) : static_cast<const bf16*>(v);
+  aa.v_row_stride = static_cast<long long>(p->hkv) * D;
+  aa.v_batch_stride = static_cast<long long>(L) * p->hkv * D;
+  aa.out = static_cast<bf16*>(out);
+  aa.lse = lse;
+  aa.L = L;
+  aa.hq = p->hq;
+  aa.hkv = p->hkv;
+  aa.w0 = plan.bif ? p->w0 : L;
+  aa.scale_log2 = scale_log2(p);
+  cudaError_t e;
+  if (D == 128)
+    e = plan.bif ? launch_attn_mma<128, true>(aa, batch, st) : launch_attn_mma<128, false>(aa, batch, st);
+  else
+    e = plan.bif ? launch_attn_mma<64, true>(aa, batch, st) : launch_attn_mma<64, false>(aa, batch, st);
+  return e == cudaSuccess ? BF_OK : BF_ERR_CUDA;
+}
+
+bf_status_t prefill_impl(bool bifocal_api, const void* q, const void* k, const void* v, int32_t dtype, int32_t batch,
+                         int32_t L, const bf_params_t* p, void* out, float* lse, void* kcache_out, void* vcache_out,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  // validate everything before the first launch
+  bf_status_t s = check_params(p, bifocal_api);
+  if (s != BF_OK) return s;
+  if (!q || !k || !v || !out) return BF_ERR_INVALID;
+  if (!aligned(out, 16)) return BF_ERR_INVALID;
+  s = prefill_rope_impl(bifocal_api, q, k, v, dtype, batch, L, p, kcache_out, vcache_out, workspace, ws_bytes, stream);
+  if (s != BF_OK) return s;
+  return prefill_attention_impl(bifocal_api, v, dtype, batch, L, p, out, lse, workspace, ws_bytes, stream);
+}
+
+// ------------------------------------------------------------------ decode
+struct DecodeLayout {
+  size_t part_o, part_ml, total;
+};
+
+DecodeLayout decode_layout(int L_max, const bf_params_t* p) {
+  DecodeLayout w{};
+  const int splits = std::min(kMaxSplits, (L_max + bf::dec::KB - 1) / bf::dec::KB);
+  w.part_o = 0;
+  w.part_ml = align256(static_cast<size_t>(splits) * p->hq * p->head_dim * 4);
+  w.total = w.part_ml + align256(static_cast<size_t>(splits) * p->hq * 2 * 4);
+  return w;
+}
+
+bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, const void* v_new, void* kcache,
+                        void* vcache, int32_t cap, int32_t L, const bf_params_t* p, void* out, float* lse,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  bf_status_t s = check_params(p, bifocal_api);
+  if (s != BF_OK) return s;
+  if (!q || !k_new || !v_new || !kcache || !vcache || !out) return BF_ERR_INVALID;
+  if (L < 1 || cap < L) return BF_ERR_INVALID;
+  if (p->hq / p->hkv > bf::dec::MAX_G) return BF_ERR_UNSUPPORTED;
+  if (!aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16))
+    return BF_ERR_INVALID;
+  const DecodeLayout lay = decode_layout(L, p);
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < lay.total) return BF_ERR_WORKSPACE;
+
+  const int D = p->head_dim;
+  const int G = bifocal_api ? factor(L, p->w_pretrained) : 1;
+  const bool bif = bifocal_api && (G > 1 || (p->flags & BF_FLAG_FORCE_BIFOCAL)) && p->w0 < L;
+  const Rope rope = make_rope(p->rope_theta, D, G);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  // 1. append the new token
+  bf::AppendArgs ap{};
+  ap.k_new = static_cast<const bf16*>(k_new);
+  ap.v_new = static_cast<const bf16*>(v_new);
+  ap.kcache = static_cast<bf16*>(kcache);
+  ap.vcache = static_cast<bf16*>(vcache);
+  ap.hkv = p->hkv;
+  ap.p = L - 1;
+  std::memcpy(ap.omega, rope.omega, sizeof(ap.omega));
+  if (D == 128)
+    bf::decode_append_kernel<128><<<p->hkv, 32, 0, st>>>(ap);
+  else
+    bf::decode_append_kernel<64><<<p->hkv, 32, 0, st>>>(ap);
+  if (cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
+
+  // 2. split-KV partials
+  bf::DecodeArgs da;
+  std::memset(&da, 0, sizeof(da));
+  if (!make_cache_map(&da.kmap, kcache, cap, p->hkv, D, bf::dec::KB) ||
+      !make_cache_map(&da.vmap, vcache, cap, p->hkv, D, bf::dec::KB))
+    return BF_ERR_CUDA;
+  const int head_groups = (p->hkv + bf::dec::HPC - 1) / bf::dec::HPC;
+  const int sms = std::max(1, sm_count());
+  const int target = std::max(1, std::min(kMaxSplits, sms / head_groups));
+  int split_len = (L + target - 1) / target;
+  split_len = (split_len + bf::dec::KB - 1) / bf::dec::KB * bf::dec::KB;
+  const int n_split = (L + split_len - 1) / split_len;
+  da.q = static_cast<const bf16*>(q);
+  da.part_o = reinterpret_cast<float*>(ws + lay.part_o);
+  da.part_ml = reinterpret_cast<float*>(ws + lay.part_ml);
+  da.L = L;
+  da.hq = p->hq;
+  da.hkv = p->hkv;
+  da.w0 = p->w0;
+  da.G = G;
+  da.mode = bifocal_api ? p->mode : 0;
+  da.bifocal = bif ? 1 : 0;
+  da.split_len = split_len;
+  da.n_split = n_split;
+  da.scale_log2 = scale_log2(p);
+  std::memcpy(da.omega, rope.omega, sizeof(da.omega));
+  std::memcpy(da.omega_long, rope.omega_long, sizeof(da.omega_long));
+  std::memcpy(da.omega_corr, rope.omega_corr, sizeof(da.omega_corr));
+  const dim3 grid(n_split, head_groups);
+  cudaError_t e;
+  if (D == 128) {
+    constexpr int smem = bf::decode_smem_bytes<128>();
+    e = cudaFuncSetAttribute(bf::decode_partial_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) bf::decode_partial_kernel<128><<<grid, (bf::dec::HPC + 1) * 32, smem, st>>>(da);
+  } else {
+    constexpr int smem = bf::decode_smem_bytes<64>();
+    e = cudaFuncSetAttribute(bf::decode_partial_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) bf::decode_partial_kernel<64><<<grid, (bf::dec::HPC + 1) * 32, smem, st>>>(da);
+  }
+  if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
+
+  // 3. combine
+  if (D == 128)
+    bf::decode_combine_kernel<128><<<p->hq, 128, 0, st>>>(da.part_o, da.part_ml, n_split, p->hq,
+                                                         static_cast<bf16*>(out), lse);
+  else
+    bf::decode_combine_kernel<64><<<p->hq, 64, 0, st>>>(da.part_o, da.part_ml, n_split, p->hq,
+                                                       static_cast<bf16*>(out), lse);
+  return cudaGetLastError() == cudaSuccess ? BF_OK : BF_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t bifocal_factor(int64_t L, int32_t w_pretrained) {
+  if (L < 0 || w_pretrained < 1) return -1;
+  return factor(L, w_pretrained);
+}
+
+size_t bifocal_prefill_workspace_size(int32_t dtype, int32_t batch, int32_t L, const bf_params_t* p) {
+  if (check_params(p, false) != BF_OK || batch < 1 || L < 1) return 0;
+  if (dtype != BF_DTYPE_BF16 && dtype != BF_DTYPE_FP32) return 0;
+  return prefill_layout(dtype, batch, L, p).total;
+}
+
+bf_status_t bifocal_prefill(const void* q, const void* k, const void* v, int32_t dtype, int32_t batch, int32_t L,
+                            const bf_params_t* p, void* out, float* lse, void* kcache_out, void* vcache_out,
+                            void* workspace, size_t ws_bytes, void* stream) {
+  return prefill_impl(true, q, k, v, dtype, batch, L, p, out, lse, kcache_out, vcache_out, workspace, ws_bytes,
+                      stream);
+}
+
+bf_status_t bifocal_prefill_rope(const void* q, const void* k, const void* v, int32_t dtype, int32_t batch,
+                                 int32_t L, const bf_params_t* p, void* kcache_out, void* vcache_out, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  return prefill_rope_impl(true, q, k, v, dtype, batch, L, p, kcache_out, vcache_out, workspace, ws_bytes, stream);
+}
+
+bf_status_t bifocal_prefill_attention(const void* v, int32_t dtype, int32_t batch, int32_t L, const bf_params_t* p,
+                                      void* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  return prefill_attention_impl(true, v, dtype, batch, L, p, out, lse, workspace, ws_bytes, stream);
+}
+
+bf_status_t rope_causal_prefill(const void* q, const void* k, const void* v, int32_t dtype, int32_t batch, int32_t L,
+                                const bf_params_t* p, void* out, float* lse, void* kcache_out, void* vcache_out,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  return prefill_impl(false, q, k, v, dtype, batch, L, p, out, lse, kcache_out, vcache_out, workspace, ws_bytes,
+                      stream);
+}
+
+size_t bifocal_decode_workspace_size(int32_t L_max, const bf_params_t* p) {
+  if (check_params(p, false) != BF_OK || L_max < 1) return 0;
+  return decode_layout(L_max, p).total;
+}
+
+bf_status_t bifocal_decode(const void* q, const void* k_new, const void* v_new, void* kcache, void* vcache,
+                           int32_t cap, int32_t L, const bf_params_t* p, void* out, float* lse, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  return decode_impl(true, q, k_new, v_new, kcache, vcache, cap, L, p, out, lse, workspace, ws_bytes, stream);
+}
+
+bf_status_t rope_causal_decode(const void* q, const void* k_new, const void* v_new, void* kcache, void* vcache,
+                               int32_t cap, int32_t L, const bf_params_t* p, void* out, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  return decode_impl(false, q, k_new, v_new, kcache, vcache, cap, L, p, out, lse, workspace, ws_bytes, stream);
+}
+
+const char* bifocal_status_string(int32_t status) {
+  switch (status) {
+    case BF_OK: return "ok";
+    case BF_ERR_INVALID: return "invalid argument";
+    case BF_ERR_UNSUPPORTED: return "unsupported configuration";
+    case BF_ERR_CUDA: return "CUDA error";
+    case BF_ERR_TIMEOUT: return "device-side wait timed out";
+    case BF_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case BF_ERR_NO_DEVICE: return "no suitable CUDA device";
+    default: return "unknown status";
+  }
+}
+
+bf_status_t bifocal_last_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return BF_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, bf::g_device_status, sizeof(int)) != cudaSuccess) return BF_ERR_CUDA;
+  if (v == 0) return BF_OK;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(bf::g_device_status, &zero, sizeof(int)) != cudaSuccess) return BF_ERR_CUDA;
+  return BF_ERR_TIMEOUT;
+}
+
+const char* bifocal_build_info(void) {
+  return "bifocal sm_100a: rope pre-pass, prefill (mma.sync m16n8k16, D=64/128), decode split-KV (TMA + mma.sync)";
+}
+
+}  // extern "C"

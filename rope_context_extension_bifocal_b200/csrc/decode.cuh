@@ -1,0 +1,327 @@
+// Single-batch decode: append, split-KV partial attention, log-sum-exp combine.
+//
+// The cache holds keys under the ORIGINAL RoPE (bf16). A cached key j that falls in
+// the long-range branch (p - j >= w0) is re-phased on the fly by the correction
+// rotation Rcorr(j) = R_long(j) R_orig(j)^-1, whose angle for pair k is
+//   j * omega_k * (1/G - 1)          (frequency interpolation)
+//   (floor(j / G) - j) * omega_k     (position aliasing)
+// (ai-feeds summary of Jet-Long, 方法 key module 3: the correction rotation of cached
+// keys; knowledge-base note, 设计原理: the near/far boundary slides during generation).
+// The rotation runs in registers on tiles staged in shared memory by TMA, so the cache
+// is read once from HBM and never rewritten. G follows the current length L, so when
+// L crosses a multiple of w_pretrained every long-range key is re-phased at once.
+//
+// Work split: CTA = (key range, up to 8 kv heads); one consumer warp per kv head and a
+// producer warp that streams 16-key stages (K and V, every head, both 64-element halves
+// of D) through a 3-deep mbarrier ring. QK^T and PV of the g = hq/hkv query rows of a
+// kv head run on mma.sync (the rows fit one m16 tile; the kernel is HBM-bound).
+// QK^T operands are fp16 (rotated query, corrected or converted cached key), PV is bf16.
+#pragma once
+#include "common.cuh"
+
+namespace bf {
+
+namespace dec {
+constexpr int KB = 16;      // keys per stage
+constexpr int NST = 3;      // stages in flight
+constexpr int HPC = 8;      // kv heads per CTA (max)
+constexpr int MAX_G = 8;    // query heads per kv head (max)
+}  // namespace dec
+
+struct DecodeArgs {
+  CUtensorMap kmap;  // cache K viewed as (d_lo 64, d_hi D/64, head hkv, key cap), box (64,1,1,KB)
+  CUtensorMap vmap;
+  const __nv_bfloat16* q;  // [hq, D] raw
+  float* part_o;           // [n_split, hq, D] unnormalised
+  float* part_ml;          // [n_split, hq, 2]: running max (log2 domain), sum
+  int L, hq, hkv, w0, G, mode, bifocal;
+  int split_len, n_split;
+  float scale_log2;
+  double omega[64];
+  double omega_long[64];  // omega / G
+  double omega_corr[64];  // omega * (1/G - 1)
+};
+
+// 128-byte swizzle of TMA SWIZZLE_128B: 16-byte chunk c of row r sits at chunk c ^ (r & 7).
+__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__((dec::HPC + 1) * 32, 1) decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
+  using namespace dec;
+  constexpr int P = D / 2;
+  constexpr int HALVES = D / 64;
+  constexpr int KC = D / 16;       // k-chunks
+  constexpr int KCP = KC / 2;      // k-chunks holding the first element of each pair
+  constexpr int DT = D / 8;        // n-tiles of O
+  constexpr uint32_t HEAD_TILE = KB * 128;                 // one head, one half: KB rows x 128 B
+  constexpr uint32_t STAGE_KV = HPC * HALVES * HEAD_TILE;  // all heads, all halves
+  constexpr int CS_STRIDE = P * 8 + 16;                    // bytes per key row of the cos/sin table
+
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sK = smem;                       // [NST][HPC][HALVES][KB][128 B]
+  uint8_t* sV = sK + NST * STAGE_KV;        // same
+  uint8_t* sCS = sV + NST * STAGE_KV;       // [2][KB][CS_STRIDE]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sCS + 2 * KB * CS_STRIDE);
+  uint64_t* empty = full + NST;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x;
+  const int head0 = blockIdx.y * HPC;
+  const int nheads = min(HPC, a.hkv - head0);
+  const int g = a.hq / a.hkv;
+  const int p = a.L - 1;
+  const int jbeg = split * a.split_len;
+  const int jend = min(a.L, jbeg + a.split_len);
+  const int nstage = (jend - jbeg + KB - 1) / KB;
+  const int local_from = a.bifocal ? max(0, a.L - a.w0) : 0;  // keys j >= local_from are local
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], nheads);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == HPC) {
+    // producer
+    if (lane == 0) {
+      prefetch_tensormap(&a.kmap);
+      prefetch_tensormap(&a.vmap);
+      const uint32_t bytes = 2u * nheads * HALVES * HEAD_TILE;
+      for (int s = 0; s < nstage; ++s) {
+        const int st = s % NST;
+        if (s >= NST && !mbar_wait(&empty[st], ((s / NST) - 1) & 1, 1)) break;
+        mbar_arrive_expect_tx(&full[st], bytes);
+        const int j0 = jbeg + s * KB;
+        for (int hh = 0; hh < nheads; ++hh)
+          for (int hf = 0; hf < HALVES; ++hf) {
+            const uint32_t off = st * STAGE_KV + (hh * HALVES + hf) * HEAD_TILE;
+            tma_load_4d(sK + off, &a.kmap, &full[st], 0, hf, head0 + hh, j0);
+            tma_load_4d(sV + off, &a.vmap, &full[st], 0, hf, head0 + hh, j0);
+          }
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers: warp w handles kv head head0 + w ----------------
+  if (warp >= nheads) return;  // fewer kv heads than warps in this CTA
+  const bool active = true;
+  const int kvh = head0 + warp;
+  const int g8 = lane >> 2, t4 = lane & 3;
+
+  // query fragments (rows 0..g-1 = the g query heads of this kv head), both branches
+  uint32_t qa_o[KC][2], qa_l[KC][2];  // a0 (k = 2t4..) and a2 (k = 8 + 2t4..); rows 8..15 are zero
+  {
+    const bool row_ok = active && g8 < g;
+    const __nv_bfloat16* qrow = a.q + static_cast<long long>(kvh * g + (row_ok ? g8 : 0)) * D;
+    const double pl = (a.mode == 0) ? static_cast<double>(p) : static_cast<double>(p / a.G);
+#pragma unroll
+    for (int kc = 0; kc < KCP; ++kc)
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub) {
+        const int d = 16 * kc + 8 * sub + 2 * t4;  // pair indices d, d + 1
+        float xo[2], yo[2], xl[2], yl[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float x = 0.f, y = 0.f;
+          if (row_ok) {
+            x = __bfloat162float(qrow[d + e]);
+            y = __bfloat162float(qrow[d + e + P]);
+          }
+          float c, s;
+          angle_cos_sin(static_cast<double>(p) * a.omega[d + e], c, s);
+          xo[e] = x * c - y * s;
+          yo[e] = y * c + x * s;
+          if (a.mode == 0)
+            angle_cos_sin(pl * a.omega_long[d + e], c, s);
+          else
+            angle_cos_sin(pl * a.omega[d + e], c, s);
+          xl[e] = x * c - y * s;
+          yl[e] = y * c + x * s;
+        }
+        qa_o[kc][sub] = pack_f16x2(xo[0], xo[1]);
+        qa_o[kc + KCP][sub] = pack_f16x2(yo[0], yo[1]);
+        qa_l[kc][sub] = pack_f16x2(xl[0], xl[1]);
+        qa_l[kc + KCP][sub] = pack_f16x2(yl[0], yl[1]);
+      }
+  }
+
+  float o[DT][4];
+#pragma unroll
+  for (int i = 0; i < DT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_r = -INFINITY, l_r = 0.f;
+  const int nthr = nheads * 32;
+  const int tid = threadIdx.x;
+
+  for (int s = 0; s < nstage; ++s) {
+    const int st = s % NST;
+    const int j0 = jbeg + s * KB;
+    const bool any_long = j0 < local_from;
+    const bool any_local = j0 + KB - 1 >= local_from;
+    // cooperative cos/sin table of the correction rotation for this stage's keys
+    uint8_t* cs = sCS + (s & 1) * KB * CS_STRIDE;
+    if (any_long) {
+      for (int idx = tid; idx < KB * P; idx += nthr) {
+        const int kk = idx / P, pr = idx % P;
+        const int j = j0 + kk;
+        const double ang = (a.mode == 0) ? static_cast<double>(j) * a.omega_corr[pr]
+                                         : static_cast<double>(j / a.G - j) * a.omega[pr];
+        float c, sn;
+        angle_cos_sin(ang, c, sn);
+        *reinterpret_cast<float2*>(cs + kk * CS_STRIDE + pr * 8) = make_float2(c, sn);
+      }
+    }
+    asm volatile("bar.sync 1, %0;\n" ::"r"(nthr));
+    if (!mbar_wait(&full[st], (s / NST) & 1, 2)) break;
+
+    const uint32_t kbase = smem_u32(sK + st * STAGE_KV + warp * HALVES * HEAD_TILE);
+    const uint32_t vbase = smem_u32(sV + st * STAGE_KV + warp * HALVES * HEAD_TILE);
+    float sc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      float so[4] = {0.f, 0.f, 0.f, 0.f}, sl[4] = {0.f, 0.f, 0.f, 0.f};
+      const int krow = nt * 8 + (lane & 7);
+      const int key_mine = nt * 8 + g8;  // key whose B elements this lane holds
+#pragma unroll
+      for (int kc = 0; kc < KCP; ++kc) {
+        // elements d = 16kc + 8*(lane>>3 & 1) + ..., and their partners d + P
+        const int e_lo = 16 * kc + 8 * ((lane >> 3) & 1) + ((lane >> 4) ? P : 0);
+        uint32_t r[4];
+        ldmatrix_x4(r, kbase + (e_lo / 64) * HEAD_TILE + sw128(krow, (e_lo % 64) / 8));
+        // r0: d = 16kc + 2t4 (+0,1); r1: d + 8; r2: d + P; r3: d + 8 + P
+        if (any_local) {
+          uint32_t a0[4] = {qa_o[kc][0], 0u, qa_o[kc][1], 0u};
+          uint32_t a1[4] = {qa_o[kc + KCP][0], 0u, qa_o[kc + KCP][1], 0u};
+          mma_f16_16816(so, a0, bf16x2_to_f16x2(r[0]), bf16x2_to_f16x2(r[1]));
+          mma_f16_16816(so, a1, bf16x2_to_f16x2(r[2]), bf16x2_to_f16x2(r[3]));
+        }
+        if (any_long) {
+          const float4 c01 = *reinterpret_cast<const float4*>(cs + key_mine * CS_STRIDE + (16 * kc + 2 * t4) * 8);
+          const float4 c89 = *reinterpret_cast<const float4*>(cs + key_mine * CS_STRIDE + (16 * kc + 8 + 2 * t4) * 8);
+          const float2 x0 = unpack_bf16x2(r[0]), x1 = unpack_bf16x2(r[1]);
+          const float2 y0 = unpack_bf16x2(r[2]), y1 = unpack_bf16x2(r[3]);
+          // pair (x, y) -> (x c - y s, y c + x s)
+          const uint32_t rx0 = pack_f16x2(x0.x * c01.x - y0.x * c01.y, x0.y * c01.z - y0.y * c01.w);
+          const uint32_t ry0 = pack_f16x2(y0.x * c01.x + x0.x * c01.y, y0.y * c01.z + x0.y * c01.w);
+          const uint32_t rx1 = pack_f16x2(x1.x * c89.x - y1.x * c89.y, x1.y * c89.z - y1.y * c89.w);
+          const uint32_t ry1 = pack_f16x2(y1.x * c89.x + x1.x * c89.y, y1.y * c89.z + x1.y * c89.w);
+          uint32_t a0[4] = {qa_l[kc][0], 0u, qa_l[kc][1], 0u};
+          uint32_t a1[4] = {qa_l[kc + KCP][0], 0u, qa_l[kc + KCP][1], 0u};
+          mma_f16_16816(sl, a0, rx0, rx1);
+          mma_f16_16816(sl, a1, ry0, ry1);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int j = j0 + nt * 8 + 2 * t4 + e;
+        float x = (j >= local_from) ? so[e] : sl[e];
+        x *= a.scale_log2;
+        if (j >= jend) x = -INFINITY;
+        sc[nt][e] = x;
+      }
+    }
+    // online softmax over row g8 (this lane holds keys 2t4, 2t4+1 of both n-tiles)
+    float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_r, mx);
+    const float ref = (m_new == -INFINITY) ? 0.f : m_new;
+    const float alpha = fast_exp2(m_r - ref);
+    m_r = m_new;
+    const float p00 = fast_exp2(sc[0][0] - ref), p01 = fast_exp2(sc[0][1] - ref);
+    const float p10 = fast_exp2(sc[1][0] - ref), p11 = fast_exp2(sc[1][1] - ref);
+    l_r = l_r * alpha + (p00 + p01 + p10 + p11);
+    uint32_t pa[4] = {pack_bf16x2(p00, p01), 0u, pack_bf16x2(p10, p11), 0u};
+#pragma unroll
+    for (int dt = 0; dt < DT; ++dt) {
+      o[dt][0] *= alpha;
+      o[dt][1] *= alpha;
+    }
+#pragma unroll
+    for (int dt = 0; dt < DT; dt += 2) {
+      // V rows = keys; ldmatrix.trans gives B[k = key][n = d]
+      const int vrow = (lane & 7) + (((lane >> 3) & 1) << 3);
+      const int dd = (dt + (lane >> 4)) * 8;  // element offset of this lane's 8-wide column block
+      uint32_t r[4];
+      ldmatrix_x4_trans(r, vbase + (dd / 64) * HEAD_TILE + sw128(vrow, (dd % 64) / 8));
+      mma_bf16_16816(o[dt], pa, r[0], r[1]);
+      mma_bf16_16816(o[dt + 1], pa, r[2], r[3]);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+
+  // partial results of this split: rows g8 < g
+  l_r += __shfl_xor_sync(0xffffffffu, l_r, 1);
+  l_r += __shfl_xor_sync(0xffffffffu, l_r, 2);
+  if (g8 < g) {
+    const int hq_idx = kvh * g + g8;
+    float* po = a.part_o + (static_cast<long long>(split) * a.hq + hq_idx) * D;
+#pragma unroll
+    for (int dt = 0; dt < DT; ++dt) *reinterpret_cast<float2*>(po + dt * 8 + 2 * t4) = make_float2(o[dt][0], o[dt][1]);
+    if (t4 == 0) {
+      float* pml = a.part_ml + (static_cast<long long>(split) * a.hq + hq_idx) * 2;
+      pml[0] = m_r;
+      pml[1] = l_r;
+    }
+  }
+}
+
+template <int D>
+constexpr int decode_smem_bytes() {
+  return 2 * dec::NST * dec::HPC * (D / 64) * dec::KB * 128 + 2 * dec::KB * (D / 2 * 8 + 16) + 2 * dec::NST * 8;
+}
+
+// Log-sum-exp merge of the split partials: one CTA per query head, one thread per d.
+template <int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ part_o,
+                                                            const float* __restrict__ part_ml, int n_split, int hq,
+                                                            __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  const int h = blockIdx.x, d = threadIdx.x;
+  float M = -INFINITY;
+  for (int s = 0; s < n_split; ++s) M = fmaxf(M, part_ml[(s * hq + h) * 2]);
+  const float ref = (M == -INFINITY) ? 0.f : M;
+  float lsum = 0.f, acc = 0.f;
+  for (int s = 0; s < n_split; ++s) {
+    const float w = exp2f(part_ml[(s * hq + h) * 2] - ref);
+    lsum += w * part_ml[(s * hq + h) * 2 + 1];
+    acc += w * part_o[(static_cast<long long>(s) * hq + h) * D + d];
+  }
+  out[h * D + d] = __float2bfloat16(acc / lsum);
+  if (lse && d == 0) lse[h] = (M + log2f(lsum)) * 0.69314718055994530942f;
+}
+
+// Append: cache row p <- (R_orig(p) k_new, v_new). One warp per kv head.
+struct AppendArgs {
+  const __nv_bfloat16* k_new;  // [hkv, D]
+  const __nv_bfloat16* v_new;  // [hkv, D]
+  __nv_bfloat16* kcache;       // [cap, hkv, D]
+  __nv_bfloat16* vcache;
+  int hkv, p;
+  double omega[64];
+};
+
+template <int D>
+__global__ void decode_append_kernel(const __grid_constant__ AppendArgs a) {
+  constexpr int P = D / 2;
+  const int h = blockIdx.x, lane = threadIdx.x;
+  const __nv_bfloat16* kr = a.k_new + h * D;
+  __nv_bfloat16* kd = a.kcache + (static_cast<long long>(a.p) * a.hkv + h) * D;
+  for (int pr = lane; pr < P; pr += 32) {
+    float c, s;
+    angle_cos_sin(static_cast<double>(a.p) * a.omega[pr], c, s);
+    const float x = __bfloat162float(kr[pr]), y = __bfloat162float(kr[pr + P]);
+    kd[pr] = __float2bfloat16(x * c - y * s);
+    kd[pr + P] = __float2bfloat16(y * c + x * s);
+  }
+  const __nv_bfloat16* vr = a.v_new + h * D;
+  __nv_bfloat16* vd = a.vcache + (static_cast<long long>(a.p) * a.hkv + h) * D;
+  for (int d = lane; d < D; d += 32) vd[d] = vr[d];
+}
+
+}  // namespace bf

@@ -1,0 +1,176 @@
+// RoPE pre-pass of the prefill: one HBM pass over the raw q and k.
+//
+// For every position p it evaluates the rotation angles once (fp64 product and range
+// reduction, see angle_cos_sin) and applies them to every head:
+//   Qo = R_orig(p) q,  Ql = R_long(p) q   -> [b, hq,  L, D] fp16 (head-major tiles)
+//   Ko = R_orig(p) k,  Kl = R_long(p) k   -> [b, hkv, L, D] fp16
+// The rotated forms are the QK^T operands. They are rounded once, to fp16 rather than
+// bf16: same tensor-core rate, 8x smaller rounding error, so a score is off by ~2e-4
+// instead of ~3e-3 (which would exceed a 1e-3 LSE bound on rows that see few keys).
+// R_orig rotates pair k by p * omega_k; R_long by p * omega_k / G (frequency
+// interpolation) or floor(p / G) * omega_k (position aliasing) - the two long-range
+// forms named by the ablation of the ai-feeds summary of Jet-Long (实验, key findings).
+// Ko is also the decode cache (keys under the original RoPE) and is written to the
+// caller's kcache in [b, L, hkv, D] when asked. fp32 inputs are rounded to bf16 here.
+#pragma once
+#include "common.cuh"
+
+namespace bf {
+
+struct PrepassArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int batch, L, hq, hkv;
+  int G;
+  int mode;       // 0 = frequency interpolation, 1 = position aliasing
+  int need_long;  // write Ql / Kl
+  __half* Qo;
+  __half* Ql;
+  __half* Ko;
+  __half* Kl;
+  __nv_bfloat16* Vb;       // bf16 copy of v in [b, L, hkv, D] (fp32 inputs only), else null
+  __nv_bfloat16* kcache;   // optional [b, L, hkv, D]
+  __nv_bfloat16* vcache;   // optional [b, L, hkv, D]
+  double omega[64];        // omega_k = theta^(-2k/D)
+  double omega_long[64];   // omega_k / G (frequency interpolation)
+};
+
+template <typename T>
+struct Vec8;  // 8 consecutive elements of T
+template <>
+struct Vec8<__nv_bfloat16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = *reinterpret_cast<const uint4*>(p); }
+  __device__ __forceinline__ float get(int i) const {
+    const uint32_t w = (&u.x)[i >> 1];
+    float2 f = unpack_bf16x2(w);
+    return (i & 1) ? f.y : f.x;
+  }
+};
+template <>
+struct Vec8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = reinterpret_cast<const float4*>(p)[0];
+    b = reinterpret_cast<const float4*>(p)[1];
+  }
+  __device__ __forceinline__ float get(int i) const {
+    const float* f = (i < 4) ? &a.x : &b.x;
+    return f[i & 3];
+  }
+};
+
+__device__ __forceinline__ void store8_f16(__half* dst, const float (&x)[8]) {
+  uint4 u;
+  u.x = pack_f16x2(x[0], x[1]);
+  u.y = pack_f16x2(x[2], x[3]);
+  u.z = pack_f16x2(x[4], x[5]);
+  u.w = pack_f16x2(x[6], x[7]);
+  *reinterpret_cast<uint4*>(dst) = u;
+}
+
+__device__ __forceinline__ void store8_bf16(__nv_bfloat16* dst, const float (&x)[8]) {
+  uint4 u;
+  u.x = pack_bf16x2(x[0], x[1]);
+  u.y = pack_bf16x2(x[2], x[3]);
+  u.z = pack_bf16x2(x[4], x[5]);
+  u.w = pack_bf16x2(x[6], x[7]);
+  *reinterpret_cast<uint4*>(dst) = u;
+}
+
+// One warp per (batch, position). Lanes form 4 groups of 8; group g handles rows
+// (heads) g, g+4, ...; lane l8 of a group owns the 8 pairs [8*l8 .. 8*l8+8) for D=128
+// (elements d and d + D/2), or 4 pairs for D=64 (then lanes 4..7 of a group idle on d).
+template <typename Tin, int D>
+__global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant__ PrepassArgs a) {
+  constexpr int P = D / 2;
+  constexpr int NPAIR = 8;               // pairs per lane slot
+  constexpr int LANES_PER_ROW = P / NPAIR;  // 8 (D=128) or 4 (D=64)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long gpos = static_cast<long long>(blockIdx.x) * 8 + warp;
+  if (gpos >= static_cast<long long>(a.batch) * a.L) return;
+  const int b = static_cast<int>(gpos / a.L);
+  const int p = static_cast<int>(gpos % a.L);
+  const int grp = lane >> 3, l8 = lane & 7;
+  if (l8 >= LANES_PER_ROW) return;
+  const int k0 = l8 * NPAIR;  // first pair index this lane owns
+
+  float co[NPAIR], so[NPAIR], cl[NPAIR], sl[NPAIR];
+  const double pl = (a.mode == 0) ? static_cast<double>(p) : static_cast<double>(p / a.G);
+#pragma unroll
+  for (int i = 0; i < NPAIR; ++i) {
+    angle_cos_sin(static_cast<double>(p) * a.omega[k0 + i], co[i], so[i]);
+    if (a.need_long) {
+      if (a.mode == 0)
+        angle_cos_sin(pl * a.omega_long[k0 + i], cl[i], sl[i]);
+      else
+        angle_cos_sin(pl * a.omega[k0 + i], cl[i], sl[i]);
+    } else {
+      cl[i] = co[i];
+      sl[i] = so[i];
+    }
+  }
+
+  const Tin* qb = static_cast<const Tin*>(a.q);
+  const Tin* kb = static_cast<const Tin*>(a.k);
+  const Tin* vb = static_cast<const Tin*>(a.v);
+  const int rows = a.hq + a.hkv;
+  for (int r = grp; r < rows; r += 4) {
+    const bool is_q = r < a.hq;
+    const int h = is_q ? r : r - a.hq;
+    const int H = is_q ? a.hq : a.hkv;
+    const Tin* src = (is_q ? qb : kb) + ((static_cast<long long>(b) * a.L + p) * H + h) * D;
+    Vec8<Tin> x1, x2;
+    x1.load(src + k0);
+    x2.load(src + P + k0);
+    float yo1[8], yo2[8], yl1[8], yl2[8];
+#pragma unroll
+    for (int i = 0; i < NPAIR; ++i) {
+      const float u = x1.get(i), w = x2.get(i);
+      yo1[i] = u * co[i] - w * so[i];
+      yo2[i] = w * co[i] + u * so[i];
+      yl1[i] = u * cl[i] - w * sl[i];
+      yl2[i] = w * cl[i] + u * sl[i];
+    }
+    const long long hm = ((static_cast<long long>(b) * H + h) * a.L + p) * D;  // head-major row
+    __half* dst_o = (is_q ? a.Qo : a.Ko) + hm;
+    store8_f16(dst_o + k0, yo1);
+    store8_f16(dst_o + P + k0, yo2);
+    if (a.need_long) {
+      __half* dst_l = (is_q ? a.Ql : a.Kl) + hm;
+      store8_f16(dst_l + k0, yl1);
+      store8_f16(dst_l + P + k0, yl2);
+    }
+    if (!is_q && a.kcache) {
+      __nv_bfloat16* dc = a.kcache + ((static_cast<long long>(b) * a.L + p) * a.hkv + h) * D;
+      store8_bf16(dc + k0, yo1);
+      store8_bf16(dc + P + k0, yo2);
+    }
+  }
+  // v: bf16 copy for fp32 inputs and / or the caller's vcache
+  if (a.Vb || a.vcache) {
+    for (int h = grp; h < a.hkv; h += 4) {
+      const long long off = ((static_cast<long long>(b) * a.L + p) * a.hkv + h) * D;
+      Vec8<Tin> x1, x2;
+      x1.load(vb + off + k0);
+      x2.load(vb + off + P + k0);
+      float y1[8], y2[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        y1[i] = x1.get(i);
+        y2[i] = x2.get(i);
+      }
+      if (a.Vb) {
+        store8_bf16(a.Vb + off + k0, y1);
+        store8_bf16(a.Vb + off + P + k0, y2);
+      }
+      if (a.vcache) {
+        store8_bf16(a.vcache + off + k0, y1);
+        store8_bf16(a.vcache + off + P + k0, y2);
+      }
+    }
+  }
+}
+
+}  // namespace bf
