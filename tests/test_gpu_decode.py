@@ -15,6 +15,10 @@ from tests.gpu_helpers import assert_close
 pytestmark = pytest.mark.gpu
 
 
+def bf16_round(x):
+    return torch.from_numpy(np.asarray(x, dtype=np.float64)).to(torch.bfloat16).double().numpy()
+
+
 def session(w: si.DecodeWorkload, check, plain=False, prefix=None, cap=None, steps=None):
     stream = si.DecodeStream(w, prefix_len=prefix, capacity=cap)
     prefix, cap = stream.prefix_len, stream.capacity
@@ -39,7 +43,8 @@ def session(w: si.DecodeWorkload, check, plain=False, prefix=None, cap=None, ste
         else:
             out, lse = bfl.bifocal_decode(q.cuda(), kn.cuda(), vn.cuda(), kcache, vcache, L, w0=w.w0,
                                           w_pretrained=w.w_pretrained, theta=w.theta, mode=w.mode)
-        ref_k[p] = R.rope_keys_for_cache(kn[None].float().double().numpy(), w.theta, start=p)[0]
+        # the cache stores bf16: round the oracle's own fp64 key to the storage format
+        ref_k[p] = bf16_round(R.rope_keys_for_cache(kn[None].float().double().numpy(), w.theta, start=p)[0])
         ref_v[p] = vn.float().double().numpy()
         if t in check:
             w0 = L if plain else w.w0
