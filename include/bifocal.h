@@ -69,6 +69,8 @@ typedef enum { BF_DTYPE_BF16 = 0, BF_DTYPE_FP32 = 1 } bf_dtype_t;
 
 /* flags */
 #define BF_FLAG_FORCE_BIFOCAL 1 /* run the two-branch kernel even when G == 1 or w0 >= L (results are equal) */
+#define BF_FLAG_MMA_SYNC 2      /* prefill, D = 128: use the warp-level mma.sync kernel instead of tcgen05
+                                   (comparison only; D = 64 always uses it) */
 
 typedef struct {
   int32_t hq;           /* query heads; hq % hkv == 0; query head h reads kv head h / (hq / hkv) */

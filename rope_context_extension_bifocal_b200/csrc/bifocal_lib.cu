@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill_mma.cuh"
+#include "prefill_tc.cuh"
 #include "rope_prepass.cuh"
 
 namespace {
@@ -98,6 +99,32 @@ bool make_cache_map(CUtensorMap* map, const void* base, int cap, int hkv, int D,
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Rotated key forms [rows = b*hkv][L][128] fp16, box (64, 128, 1), 128B swizzle.
+bool make_k_map(CUtensorMap* map, const void* base, int L, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(L) * 256};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// V [b][L][hkv][128] bf16, box (64, 1, 128, 1), 128B swizzle: one 128-byte row per key.
+bool make_v_map(CUtensorMap* map, const void* base, int L, int hkv, int batch) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(hkv), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[3] = {256, static_cast<cuuint64_t>(hkv) * 256, static_cast<cuuint64_t>(L) * hkv * 256};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 // ------------------------------------------------------------------ prefill
 struct PrefillLayout {
@@ -234,10 +261,37 @@ bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtyp
   aa.w0 = plan.bif ? p->w0 : L;
   aa.scale_log2 = scale_log2(p);
   cudaError_t e;
-  if (D == 128)
+  if (D == 128 && !(p->flags & BF_FLAG_MMA_SYNC)) {
+    // tcgen05 path
+    bf::TcArgs ta;
+    std::memset(&ta, 0, sizeof(ta));
+    if (!make_k_map(&ta.ko_map, aa.Ko, L, batch * p->hkv) || !make_k_map(&ta.kl_map, aa.Kl, L, batch * p->hkv) ||
+        !make_v_map(&ta.v_map, aa.V, L, p->hkv, batch))
+      return BF_ERR_CUDA;
+    ta.Qo = aa.Qo;
+    ta.Ql = aa.Ql;
+    ta.out = aa.out;
+    ta.lse = aa.lse;
+    ta.L = L;
+    ta.hq = p->hq;
+    ta.hkv = p->hkv;
+    ta.batch = batch;
+    ta.w0 = aa.w0;
+    ta.scale_log2 = aa.scale_log2;
+    constexpr int smem = bf::attn_tc_smem_bytes();
+    const long long n_cta = static_cast<long long>((L + bf::tc::BM - 1) / bf::tc::BM) * p->hq * batch;
+    if (n_cta > 0x7fffffffLL) return BF_ERR_UNSUPPORTED;
+    auto kern = plan.bif ? bf::attn_tc_kernel<true> : bf::attn_tc_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) {
+      kern<<<static_cast<unsigned>(n_cta), bf::tc::NTHREADS, smem, st>>>(ta);
+      e = cudaGetLastError();
+    }
+  } else if (D == 128) {
     e = plan.bif ? launch_attn_mma<128, true>(aa, batch, st) : launch_attn_mma<128, false>(aa, batch, st);
-  else
+  } else {
     e = plan.bif ? launch_attn_mma<64, true>(aa, batch, st) : launch_attn_mma<64, false>(aa, batch, st);
+  }
   return e == cudaSuccess ? BF_OK : BF_ERR_CUDA;
 }
 
@@ -261,7 +315,8 @@ struct DecodeLayout {
 
 DecodeLayout decode_layout(int L_max, const bf_params_t* p) {
   DecodeLayout w{};
-  const int splits = std::min(kMaxSplits, (L_max + bf::dec::KB - 1) / bf::dec::KB);
+  // two partials (one per consumer warp of a kv head) per CTA split
+  const int splits = 2 * std::min(kMaxSplits, (L_max + bf::dec::KB - 1) / bf::dec::KB);
   w.part_o = 0;
   w.part_ml = align256(static_cast<size_t>(splits) * p->hq * p->head_dim * 4);
   w.total = w.part_ml + align256(static_cast<size_t>(splits) * p->hq * 2 * 4);
@@ -336,20 +391,20 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
   if (D == 128) {
     constexpr int smem = bf::decode_smem_bytes<128>();
     e = cudaFuncSetAttribute(bf::decode_partial_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) bf::decode_partial_kernel<128><<<grid, (bf::dec::HPC + 1) * 32, smem, st>>>(da);
+    if (e == cudaSuccess) bf::decode_partial_kernel<128><<<grid, bf::decode_threads<128>(), smem, st>>>(da);
   } else {
     constexpr int smem = bf::decode_smem_bytes<64>();
     e = cudaFuncSetAttribute(bf::decode_partial_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) bf::decode_partial_kernel<64><<<grid, (bf::dec::HPC + 1) * 32, smem, st>>>(da);
+    if (e == cudaSuccess) bf::decode_partial_kernel<64><<<grid, bf::decode_threads<64>(), smem, st>>>(da);
   }
   if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
 
   // 3. combine
   if (D == 128)
-    bf::decode_combine_kernel<128><<<p->hq, 128, 0, st>>>(da.part_o, da.part_ml, n_split, p->hq,
+    bf::decode_combine_kernel<128><<<p->hq, 128, 0, st>>>(da.part_o, da.part_ml, 2 * n_split, p->hq,
                                                          static_cast<bf16*>(out), lse);
   else
-    bf::decode_combine_kernel<64><<<p->hq, 64, 0, st>>>(da.part_o, da.part_ml, n_split, p->hq,
+    bf::decode_combine_kernel<64><<<p->hq, 64, 0, st>>>(da.part_o, da.part_ml, 2 * n_split, p->hq,
                                                        static_cast<bf16*>(out), lse);
   return cudaGetLastError() == cudaSuccess ? BF_OK : BF_ERR_CUDA;
 }
@@ -435,7 +490,8 @@ bf_status_t bifocal_last_device_error(void* stream) {
 }
 
 const char* bifocal_build_info(void) {
-  return "bifocal sm_100a: rope pre-pass, prefill (mma.sync m16n8k16, D=64/128), decode split-KV (TMA + mma.sync)";
+  return "bifocal sm_100a: rope pass; prefill D=128 tcgen05/TMEM/TMA (D=64 and BF_FLAG_MMA_SYNC: mma.sync); "
+         "decode split-KV (TMA + mma.sync)";
 }
 
 }  // extern "C"

@@ -80,6 +80,14 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// m16n8k8, bf16: a0 = A[g][2t..2t+1], a1 = A[g+8][2t..2t+1]; b0 = B[2t..2t+1][g]
+__device__ __forceinline__ void mma_bf16_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t smem_addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -152,6 +160,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, int whe
     if (mbar_try_wait(bar, phase)) return true;
     if ((it & 63) == 0 && global_ns() - t0 > 2000000000ull) break;
   }
+  report_timeout(where);
+  return false;
+}
+
+// Same, but also gives up as soon as *abort is set (by any warp of the CTA), and sets it
+// on its own timeout, so that one expired wait makes every later wait of the CTA return.
+__device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t phase, int where, volatile int* abort) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, phase)) return true;
+    if ((it & 63) == 0) {
+      if (*abort) return false;
+      if (global_ns() - t0 > 2000000000ull) break;
+    }
+  }
+  *abort = 1;
   report_timeout(where);
   return false;
 }

@@ -11,10 +11,12 @@
 // is read once from HBM and never rewritten. G follows the current length L, so when
 // L crosses a multiple of w_pretrained every long-range key is re-phased at once.
 //
-// Work split: CTA = (key range, up to 8 kv heads); one consumer warp per kv head and a
-// producer warp that streams 16-key stages (K and V, every head, both 64-element halves
-// of D) through a 3-deep mbarrier ring. QK^T and PV of the g = hq/hkv query rows of a
-// kv head run on mma.sync (the rows fit one m16 tile; the kernel is HBM-bound).
+// Work split: CTA = (key range, up to 8 kv heads); a producer warp streams 16-key stages
+// (K and V, every head, both 64-element halves of D) through a 3-deep mbarrier ring, and
+// two consumer warps per kv head each take one 8-key n-tile of every stage, keeping their
+// own online softmax (each warp is a split of its own for the combine). QK^T of the
+// g = hq/hkv query rows runs on mma.sync m16n8k16 (rows in M); PV runs transposed,
+// O^T = V^T P^T on m16n8k8, so the query rows sit in N and the accumulator is D x 8.
 // QK^T operands are fp16 (rotated query, corrected or converted cached key), PV is bf16.
 #pragma once
 #include "common.cuh"
@@ -23,7 +25,7 @@ namespace bf {
 
 namespace dec {
 constexpr int KB = 16;      // keys per stage
-constexpr int NST = 3;      // stages in flight
+constexpr int NST = 2;      // stages in flight (2 x 64 KB per SM is ample for HBM latency)
 constexpr int HPC = 8;      // kv heads per CTA (max)
 constexpr int MAX_G = 8;    // query heads per kv head (max)
 }  // namespace dec
@@ -48,53 +50,56 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
 }
 
 template <int D>
-__global__ void __launch_bounds__((dec::HPC + 1) * 32, 1) decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
   using namespace dec;
   constexpr int P = D / 2;
   constexpr int HALVES = D / 64;
-  constexpr int KC = D / 16;       // k-chunks
+  constexpr int KC = D / 16;       // k-chunks of QK^T
   constexpr int KCP = KC / 2;      // k-chunks holding the first element of each pair
-  constexpr int DT = D / 8;        // n-tiles of O
+  constexpr int MT = D / 16;       // m-tiles of O^T (16 d-values each)
   constexpr uint32_t HEAD_TILE = KB * 128;                 // one head, one half: KB rows x 128 B
   constexpr uint32_t STAGE_KV = HPC * HALVES * HEAD_TILE;  // all heads, all halves
-  constexpr int CS_STRIDE = P * 8 + 16;                    // bytes per key row of the cos/sin table
+  constexpr int CS_STRIDE = P * 8 + 64;  // bytes per key row of the cos/sin table (pad: rows 16 banks apart)
 
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sK = smem;                       // [NST][HPC][HALVES][KB][128 B]
   uint8_t* sV = sK + NST * STAGE_KV;        // same
   uint8_t* sCS = sV + NST * STAGE_KV;       // [2][KB][CS_STRIDE]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sCS + 2 * KB * CS_STRIDE);
+  uint4* sQA = reinterpret_cast<uint4*>(sCS + 2 * KB * CS_STRIDE);  // [HPC][KC][32 lanes] query fragments
+  uint64_t* full = reinterpret_cast<uint64_t*>(sQA + HPC * KC * 32);
   uint64_t* empty = full + NST;
+  __shared__ int s_abort;  // set when a bounded wait expires: later waits return at once
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
   const int head0 = blockIdx.y * HPC;
   const int nheads = min(HPC, a.hkv - head0);
   const int g = a.hq / a.hkv;
   const int p = a.L - 1;
-  const int jbeg = split * a.split_len;
+  const int jbeg = blockIdx.x * a.split_len;
   const int jend = min(a.L, jbeg + a.split_len);
   const int nstage = (jend - jbeg + KB - 1) / KB;
   const int local_from = a.bifocal ? max(0, a.L - a.w0) : 0;  // keys j >= local_from are local
+  const int nconsumers = 2 * nheads;  // two warps per kv head, one 8-key n-tile of each stage each
 
   if (threadIdx.x == 0) {
+    s_abort = 0;
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], nheads);
+      mbar_init(&empty[s], nconsumers);
     }
     fence_barrier_init();
   }
   __syncthreads();
 
-  if (warp == HPC) {
-    // producer
+  if (warp == 2 * HPC) {
+    // producer: one elected lane streams the stages
     if (lane == 0) {
       prefetch_tensormap(&a.kmap);
       prefetch_tensormap(&a.vmap);
       const uint32_t bytes = 2u * nheads * HALVES * HEAD_TILE;
       for (int s = 0; s < nstage; ++s) {
         const int st = s % NST;
-        if (s >= NST && !mbar_wait(&empty[st], ((s / NST) - 1) & 1, 1)) break;
+        if (s >= NST && !mbar_wait_abortable(&empty[st], ((s / NST) - 1) & 1, 1, &s_abort)) break;
         mbar_arrive_expect_tx(&full[st], bytes);
         const int j0 = jbeg + s * KB;
         for (int hh = 0; hh < nheads; ++hh)
@@ -107,21 +112,25 @@ __global__ void __launch_bounds__((dec::HPC + 1) * 32, 1) decode_partial_kernel(
     }
     return;
   }
+  if (warp >= nconsumers) return;  // fewer kv heads than warp pairs in this CTA
 
-  // ---------------- consumers: warp w handles kv head head0 + w ----------------
-  if (warp >= nheads) return;  // fewer kv heads than warps in this CTA
-  const bool active = true;
-  const int kvh = head0 + warp;
+  // ---------------- consumers: warp pair (2h, 2h+1) handles kv head head0 + h ----------------
+  const int hl = warp >> 1, nt = warp & 1;  // local kv head, n-tile (keys 8nt..8nt+7 of each stage)
+  const int kvh = head0 + hl;
   const int g8 = lane >> 2, t4 = lane & 3;
 
-  // query fragments (rows 0..g-1 = the g query heads of this kv head), both branches
-  uint32_t qa_o[KC][2], qa_l[KC][2];  // a0 (k = 2t4..) and a2 (k = 8 + 2t4..); rows 8..15 are zero
-  {
-    const bool row_ok = active && g8 < g;
+  // Query fragments (rows 0..g-1 = the g query heads of this kv head) under both RoPE
+  // forms, fp16, in the m16n8k16 A layout: per k-chunk pair (kc, kc + KC/2) a lane holds
+  // {orig a0, orig a2} of chunk kc and chunk kc + KC/2 ... stored as two uint4 per kc:
+  // sQA[hl][kc][lane] = {o(kc).a0, o(kc).a2, l(kc).a0, l(kc).a2}, kc < KC (rows 8..15 are zero).
+  if (nt == 0) {
+    const bool row_ok = g8 < g;
     const __nv_bfloat16* qrow = a.q + static_cast<long long>(kvh * g + (row_ok ? g8 : 0)) * D;
     const double pl = (a.mode == 0) ? static_cast<double>(p) : static_cast<double>(p / a.G);
+    uint4* dst = sQA + hl * KC * 32;
 #pragma unroll
-    for (int kc = 0; kc < KCP; ++kc)
+    for (int kc = 0; kc < KCP; ++kc) {
+      uint32_t fo[2][2], fl[2][2];  // [first/second element of the pair][sub]
 #pragma unroll
       for (int sub = 0; sub < 2; ++sub) {
         const int d = 16 * kc + 8 * sub + 2 * t4;  // pair indices d, d + 1
@@ -133,36 +142,43 @@ __global__ void __launch_bounds__((dec::HPC + 1) * 32, 1) decode_partial_kernel(
             x = __bfloat162float(qrow[d + e]);
             y = __bfloat162float(qrow[d + e + P]);
           }
-          float c, s;
-          angle_cos_sin(static_cast<double>(p) * a.omega[d + e], c, s);
-          xo[e] = x * c - y * s;
-          yo[e] = y * c + x * s;
+          float c, sn;
+          angle_cos_sin(static_cast<double>(p) * a.omega[d + e], c, sn);
+          xo[e] = x * c - y * sn;
+          yo[e] = y * c + x * sn;
           if (a.mode == 0)
-            angle_cos_sin(pl * a.omega_long[d + e], c, s);
+            angle_cos_sin(pl * a.omega_long[d + e], c, sn);
           else
-            angle_cos_sin(pl * a.omega[d + e], c, s);
-          xl[e] = x * c - y * s;
-          yl[e] = y * c + x * s;
+            angle_cos_sin(pl * a.omega[d + e], c, sn);
+          xl[e] = x * c - y * sn;
+          yl[e] = y * c + x * sn;
         }
-        qa_o[kc][sub] = pack_f16x2(xo[0], xo[1]);
-        qa_o[kc + KCP][sub] = pack_f16x2(yo[0], yo[1]);
-        qa_l[kc][sub] = pack_f16x2(xl[0], xl[1]);
-        qa_l[kc + KCP][sub] = pack_f16x2(yl[0], yl[1]);
+        fo[0][sub] = pack_f16x2(xo[0], xo[1]);
+        fo[1][sub] = pack_f16x2(yo[0], yo[1]);
+        fl[0][sub] = pack_f16x2(xl[0], xl[1]);
+        fl[1][sub] = pack_f16x2(yl[0], yl[1]);
       }
+      dst[(2 * kc) * 32 + lane] = make_uint4(fo[0][0], fo[0][1], fl[0][0], fl[0][1]);      // chunk kc
+      dst[(2 * kc + 1) * 32 + lane] = make_uint4(fo[1][0], fo[1][1], fl[1][0], fl[1][1]);  // chunk kc + KC/2
+    }
   }
+  const uint4* qfrag = sQA + hl * KC * 32;
 
-  float o[DT][4];
+  // O^T [D x 8 query rows]: o[mt][0..1] = d = 16mt + g8, rows 2t4, 2t4+1; o[mt][2..3] = d + 8
+  float o[MT][4];
 #pragma unroll
-  for (int i = 0; i < DT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m_r = -INFINITY, l_r = 0.f;
-  const int nthr = nheads * 32;
+  for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_r = -INFINITY, l_r = 0.f;  // softmax state of query row g8 (S layout)
+  const int nthr = nconsumers * 32;
   const int tid = threadIdx.x;
 
   for (int s = 0; s < nstage; ++s) {
     const int st = s % NST;
     const int j0 = jbeg + s * KB;
     const bool any_long = j0 < local_from;
-    const bool any_local = j0 + KB - 1 >= local_from;
+    const int jt = j0 + nt * 8;  // first key of this warp's n-tile
+    const bool tile_long = jt < local_from;
+    const bool tile_local = jt + 7 >= local_from;
     // cooperative cos/sin table of the correction rotation for this stage's keys
     uint8_t* cs = sCS + (s & 1) * KB * CS_STRIDE;
     if (any_long) {
@@ -176,105 +192,125 @@ __global__ void __launch_bounds__((dec::HPC + 1) * 32, 1) decode_partial_kernel(
         *reinterpret_cast<float2*>(cs + kk * CS_STRIDE + pr * 8) = make_float2(c, sn);
       }
     }
-    asm volatile("bar.sync 1, %0;\n" ::"r"(nthr));
-    if (!mbar_wait(&full[st], (s / NST) & 1, 2)) break;
+    asm volatile("bar.sync 1, %0;\n" ::"r"(nthr));  // also publishes the query fragments
+    // after an expired wait every warp still takes part in the barriers but computes nothing
+    if (!mbar_wait_abortable(&full[st], (s / NST) & 1, 2, &s_abort)) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+      continue;
+    }
 
-    const uint32_t kbase = smem_u32(sK + st * STAGE_KV + warp * HALVES * HEAD_TILE);
-    const uint32_t vbase = smem_u32(sV + st * STAGE_KV + warp * HALVES * HEAD_TILE);
-    float sc[2][4];
+    const uint32_t kbase = smem_u32(sK + st * STAGE_KV + hl * HALVES * HEAD_TILE);
+    const uint32_t vbase = smem_u32(sV + st * STAGE_KV + hl * HALVES * HEAD_TILE);
+    float so[4] = {0.f, 0.f, 0.f, 0.f}, sl[4] = {0.f, 0.f, 0.f, 0.f};
+    const int krow = nt * 8 + (lane & 7);
+    const int key_mine = nt * 8 + g8;  // key whose B elements this lane holds
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      float so[4] = {0.f, 0.f, 0.f, 0.f}, sl[4] = {0.f, 0.f, 0.f, 0.f};
-      const int krow = nt * 8 + (lane & 7);
-      const int key_mine = nt * 8 + g8;  // key whose B elements this lane holds
-#pragma unroll
-      for (int kc = 0; kc < KCP; ++kc) {
-        // elements d = 16kc + 8*(lane>>3 & 1) + ..., and their partners d + P
-        const int e_lo = 16 * kc + 8 * ((lane >> 3) & 1) + ((lane >> 4) ? P : 0);
-        uint32_t r[4];
-        ldmatrix_x4(r, kbase + (e_lo / 64) * HEAD_TILE + sw128(krow, (e_lo % 64) / 8));
-        // r0: d = 16kc + 2t4 (+0,1); r1: d + 8; r2: d + P; r3: d + 8 + P
-        if (any_local) {
-          uint32_t a0[4] = {qa_o[kc][0], 0u, qa_o[kc][1], 0u};
-          uint32_t a1[4] = {qa_o[kc + KCP][0], 0u, qa_o[kc + KCP][1], 0u};
-          mma_f16_16816(so, a0, bf16x2_to_f16x2(r[0]), bf16x2_to_f16x2(r[1]));
-          mma_f16_16816(so, a1, bf16x2_to_f16x2(r[2]), bf16x2_to_f16x2(r[3]));
-        }
-        if (any_long) {
-          const float4 c01 = *reinterpret_cast<const float4*>(cs + key_mine * CS_STRIDE + (16 * kc + 2 * t4) * 8);
-          const float4 c89 = *reinterpret_cast<const float4*>(cs + key_mine * CS_STRIDE + (16 * kc + 8 + 2 * t4) * 8);
-          const float2 x0 = unpack_bf16x2(r[0]), x1 = unpack_bf16x2(r[1]);
-          const float2 y0 = unpack_bf16x2(r[2]), y1 = unpack_bf16x2(r[3]);
-          // pair (x, y) -> (x c - y s, y c + x s)
-          const uint32_t rx0 = pack_f16x2(x0.x * c01.x - y0.x * c01.y, x0.y * c01.z - y0.y * c01.w);
-          const uint32_t ry0 = pack_f16x2(y0.x * c01.x + x0.x * c01.y, y0.y * c01.z + x0.y * c01.w);
-          const uint32_t rx1 = pack_f16x2(x1.x * c89.x - y1.x * c89.y, x1.y * c89.z - y1.y * c89.w);
-          const uint32_t ry1 = pack_f16x2(y1.x * c89.x + x1.x * c89.y, y1.y * c89.z + x1.y * c89.w);
-          uint32_t a0[4] = {qa_l[kc][0], 0u, qa_l[kc][1], 0u};
-          uint32_t a1[4] = {qa_l[kc + KCP][0], 0u, qa_l[kc + KCP][1], 0u};
-          mma_f16_16816(sl, a0, rx0, rx1);
-          mma_f16_16816(sl, a1, ry0, ry1);
-        }
+    for (int kc = 0; kc < KCP; ++kc) {
+      // lanes 0-7: d = 16kc.., 8-15: d + 8, 16-23: d + P, 24-31: d + 8 + P
+      const int e_lo = 16 * kc + 8 * ((lane >> 3) & 1) + ((lane >> 4) ? P : 0);
+      uint32_t r[4];
+      ldmatrix_x4(r, kbase + (e_lo / 64) * HEAD_TILE + sw128(krow, (e_lo % 64) / 8));
+      const uint4 qf0 = qfrag[(2 * kc) * 32 + lane], qf1 = qfrag[(2 * kc + 1) * 32 + lane];
+      if (tile_local) {
+        uint32_t a0[4] = {qf0.x, 0u, qf0.y, 0u};
+        uint32_t a1[4] = {qf1.x, 0u, qf1.y, 0u};
+        mma_f16_16816(so, a0, bf16x2_to_f16x2(r[0]), bf16x2_to_f16x2(r[1]));
+        mma_f16_16816(so, a1, bf16x2_to_f16x2(r[2]), bf16x2_to_f16x2(r[3]));
       }
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int j = j0 + nt * 8 + 2 * t4 + e;
-        float x = (j >= local_from) ? so[e] : sl[e];
-        x *= a.scale_log2;
-        if (j >= jend) x = -INFINITY;
-        sc[nt][e] = x;
+      if (tile_long) {
+        const float4 c01 = *reinterpret_cast<const float4*>(cs + key_mine * CS_STRIDE + (16 * kc + 2 * t4) * 8);
+        const float4 c89 = *reinterpret_cast<const float4*>(cs + key_mine * CS_STRIDE + (16 * kc + 8 + 2 * t4) * 8);
+        const float2 x0 = unpack_bf16x2(r[0]), x1 = unpack_bf16x2(r[1]);
+        const float2 y0 = unpack_bf16x2(r[2]), y1 = unpack_bf16x2(r[3]);
+        // pair (x, y) -> (x c - y s, y c + x s)
+        const uint32_t rx0 = pack_f16x2(x0.x * c01.x - y0.x * c01.y, x0.y * c01.z - y0.y * c01.w);
+        const uint32_t ry0 = pack_f16x2(y0.x * c01.x + x0.x * c01.y, y0.y * c01.z + x0.y * c01.w);
+        const uint32_t rx1 = pack_f16x2(x1.x * c89.x - y1.x * c89.y, x1.y * c89.z - y1.y * c89.w);
+        const uint32_t ry1 = pack_f16x2(y1.x * c89.x + x1.x * c89.y, y1.y * c89.z + x1.y * c89.w);
+        uint32_t a0[4] = {qf0.z, 0u, qf0.w, 0u};
+        uint32_t a1[4] = {qf1.z, 0u, qf1.w, 0u};
+        mma_f16_16816(sl, a0, rx0, rx1);
+        mma_f16_16816(sl, a1, ry0, ry1);
       }
     }
-    // online softmax over row g8 (this lane holds keys 2t4, 2t4+1 of both n-tiles)
-    float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+    // merged scores of row g8 for keys jt + 2t4 + {0, 1}
+    float sc[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int j = jt + 2 * t4 + e;
+      float x = (j >= local_from) ? so[e] : sl[e];
+      x *= a.scale_log2;
+      if (j >= jend) x = -INFINITY;
+      sc[e] = x;
+    }
+    // online softmax of row g8 over this n-tile
+    float mx = fmaxf(sc[0], sc[1]);
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     const float m_new = fmaxf(m_r, mx);
     const float ref = (m_new == -INFINITY) ? 0.f : m_new;
     const float alpha = fast_exp2(m_r - ref);
     m_r = m_new;
-    const float p00 = fast_exp2(sc[0][0] - ref), p01 = fast_exp2(sc[0][1] - ref);
-    const float p10 = fast_exp2(sc[1][0] - ref), p11 = fast_exp2(sc[1][1] - ref);
-    l_r = l_r * alpha + (p00 + p01 + p10 + p11);
-    uint32_t pa[4] = {pack_bf16x2(p00, p01), 0u, pack_bf16x2(p10, p11), 0u};
+    const float p0 = fast_exp2(sc[0] - ref), p1 = fast_exp2(sc[1] - ref);
+    l_r = l_r * alpha + (p0 + p1);
+    // O^T columns are query rows 2t4 and 2t4 + 1: fetch their rescale factors
+    const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * t4);
+    const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * t4 + 4);
+    // B = P^T: b0 = P[row g8][keys 2t4, 2t4 + 1] is exactly this lane's score pair
+    const uint32_t pb = pack_bf16x2(p0, p1);
 #pragma unroll
-    for (int dt = 0; dt < DT; ++dt) {
-      o[dt][0] *= alpha;
-      o[dt][1] *= alpha;
+    for (int mt = 0; mt < MT; ++mt) {
+      o[mt][0] *= al0;
+      o[mt][1] *= al1;
+      o[mt][2] *= al0;
+      o[mt][3] *= al1;
     }
 #pragma unroll
-    for (int dt = 0; dt < DT; dt += 2) {
-      // V rows = keys; ldmatrix.trans gives B[k = key][n = d]
-      const int vrow = (lane & 7) + (((lane >> 3) & 1) << 3);
-      const int dd = (dt + (lane >> 4)) * 8;  // element offset of this lane's 8-wide column block
+    for (int mt = 0; mt < MT; mt += 2) {
+      // A = V^T: four 8x8 blocks (keys x d) of d-blocks 2mt .. 2mt+3, transposed by ldmatrix
+      const int db = 2 * mt + (lane >> 3);
       uint32_t r[4];
-      ldmatrix_x4_trans(r, vbase + (dd / 64) * HEAD_TILE + sw128(vrow, (dd % 64) / 8));
-      mma_bf16_16816(o[dt], pa, r[0], r[1]);
-      mma_bf16_16816(o[dt + 1], pa, r[2], r[3]);
+      ldmatrix_x4_trans(r, vbase + (db / 8) * HEAD_TILE + sw128(krow, db % 8));
+      mma_bf16_1688(o[mt], r[0], r[1], pb);
+      mma_bf16_1688(o[mt + 1], r[2], r[3], pb);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
   }
 
-  // partial results of this split: rows g8 < g
+  // partial results of this warp (its own split): rows < g
   l_r += __shfl_xor_sync(0xffffffffu, l_r, 1);
   l_r += __shfl_xor_sync(0xffffffffu, l_r, 2);
-  if (g8 < g) {
-    const int hq_idx = kvh * g + g8;
-    float* po = a.part_o + (static_cast<long long>(split) * a.hq + hq_idx) * D;
+  const long long split = static_cast<long long>(blockIdx.x) * 2 + nt;
 #pragma unroll
-    for (int dt = 0; dt < DT; ++dt) *reinterpret_cast<float2*>(po + dt * 8 + 2 * t4) = make_float2(o[dt][0], o[dt][1]);
-    if (t4 == 0) {
-      float* pml = a.part_ml + (static_cast<long long>(split) * a.hq + hq_idx) * 2;
-      pml[0] = m_r;
-      pml[1] = l_r;
+  for (int e = 0; e < 2; ++e) {
+    const int row = 2 * t4 + e;
+    if (row < g) {
+      float* po = a.part_o + (split * a.hq + kvh * g + row) * D;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        po[16 * mt + g8] = o[mt][e];
+        po[16 * mt + g8 + 8] = o[mt][2 + e];
+      }
     }
+  }
+  if (t4 == 0 && g8 < g) {
+    float* pml = a.part_ml + (split * a.hq + kvh * g + g8) * 2;
+    pml[0] = m_r;
+    pml[1] = l_r;
   }
 }
 
 template <int D>
 constexpr int decode_smem_bytes() {
-  return 2 * dec::NST * dec::HPC * (D / 64) * dec::KB * 128 + 2 * dec::KB * (D / 2 * 8 + 16) + 2 * dec::NST * 8;
+  return 2 * dec::NST * dec::HPC * (D / 64) * dec::KB * 128 + 2 * dec::KB * (D / 2 * 8 + 64) +
+         dec::HPC * (D / 16) * 32 * 16 + 2 * dec::NST * 8;
+}
+
+template <int D>
+constexpr int decode_threads() {
+  return (2 * dec::HPC + 1) * 32;
 }
 
 // Log-sum-exp merge of the split partials: one CTA per query head, one thread per d.

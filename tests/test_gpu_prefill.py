@@ -61,6 +61,23 @@ def test_edge_cases(L, hq, hkv, D, w0, w_pre, mode):
     assert_close(out.cpu().float().numpy(), lse.cpu().numpy(), ro, rl, f"L={L} w0={w0} w_pre={w_pre} {mode}")
 
 
+@pytest.mark.parametrize("L,hq,hkv,D,w0,w_pre,mode", [EDGE[2], EDGE[5], EDGE[12], EDGE[13]])
+def test_edge_cases_mma_sync_path(L, hq, hkv, D, w0, w_pre, mode):
+    # the warp-level mma.sync kernel (D = 64 path, and D = 128 on request) against the oracle
+    q, k, v = si.random_qkv(100 + L, 1, L, hq, hkv, D, "bf16")
+    out, lse, _, _ = run_prefill(q, k, v, w0, w_pre, 1e4, mode, flags=bfl.FLAG_MMA_SYNC)
+    ro, rl = R.bifocal_attention(np64(q), np64(k), np64(v), w0, w_pre, 1e4, mode)
+    assert_close(out.cpu().float().numpy(), lse.cpu().numpy(), ro, rl, f"mma.sync L={L} w0={w0} {mode}")
+
+
+def test_tcgen05_and_mma_sync_agree():
+    q, k, v = si.random_qkv(13, 1, 2000, 8, 2, 128, "bf16")
+    a, la, _, _ = run_prefill(q, k, v, 300, 512, 1e6, si.FREQ_INTERP)
+    b, lb, _, _ = run_prefill(q, k, v, 300, 512, 1e6, si.FREQ_INTERP, flags=bfl.FLAG_MMA_SYNC)
+    assert (a.float() - b.float()).abs().max().item() < 2e-2
+    assert (la - lb).abs().max().item() < 1e-3
+
+
 def test_batch_two():
     q, k, v = si.random_qkv(7, 2, 300, 4, 2, 128, "bf16")
     out, lse, _, _ = run_prefill(q, k, v, 50, 100, 1e4, si.POS_ALIAS)
