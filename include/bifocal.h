@@ -167,6 +167,10 @@ BF_API const char* bifocal_status_string(int32_t status);
  * current device. Synchronises `stream` first. Returns BF_OK, BF_ERR_TIMEOUT or BF_ERR_CUDA. */
 BF_API bf_status_t bifocal_last_device_error(void* stream);
 
+/* The raw device status word (not cleared): 0, or 1 | (site << 8) for the first bounded wait
+ * that expired, where `site` numbers the wait in the kernel source. Synchronises the device. */
+BF_API int32_t bifocal_device_status_word(void);
+
 /* Library build identification (static string): kernels compiled in and their target. */
 BF_API const char* bifocal_build_info(void);
 

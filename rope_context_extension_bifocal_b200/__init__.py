@@ -78,6 +78,7 @@ def _lib() -> ctypes.CDLL:
         L.bifocal_status_string.argtypes, L.bifocal_status_string.restype = [i32], ctypes.c_char_p
         L.bifocal_last_device_error.argtypes, L.bifocal_last_device_error.restype = [vp], i32
         L.bifocal_build_info.argtypes, L.bifocal_build_info.restype = [], ctypes.c_char_p
+        L.bifocal_device_status_word.argtypes, L.bifocal_device_status_word.restype = [], i32
         _LIB = L
     return _LIB
 
@@ -229,6 +230,11 @@ def rope_causal_decode(q, k_new, v_new, kcache, vcache, L: int, *, theta: float,
                        want_lse: bool = True, out=None, workspace=None, stream=None):
     p = make_params(q.shape[0], k_new.shape[0], q.shape[1], 0, 1, theta, FREQ_INTERP, scale, 0)
     return _decode("rope_causal_decode", q, k_new, v_new, kcache, vcache, L, p, want_lse, out, workspace, stream)
+
+
+def device_status_word() -> int:
+    """Raw device status word: 0, or 1 | (site << 8) of the first expired bounded wait."""
+    return int(_lib().bifocal_device_status_word())
 
 
 def last_device_error(stream=None) -> int:

@@ -489,6 +489,13 @@ bf_status_t bifocal_last_device_error(void* stream) {
   return BF_ERR_TIMEOUT;
 }
 
+int32_t bifocal_device_status_word(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, bf::g_device_status, sizeof(int)) != cudaSuccess) return -1;
+  return v;
+}
+
 const char* bifocal_build_info(void) {
   return "bifocal sm_100a: rope pass; prefill D=128 tcgen05/TMEM/TMA (D=64 and BF_FLAG_MMA_SYNC: mma.sync); "
          "decode split-KV (TMA + mma.sync)";

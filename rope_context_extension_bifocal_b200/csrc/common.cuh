@@ -181,6 +181,17 @@ __device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t phas
   return false;
 }
 
+// Warp-level wait: lane 0 polls (bounded, abortable), then every lane takes its own
+// acquire with one try_wait on the (now completed) phase. Returns a warp-uniform result.
+// The caller guarantees the barrier cannot advance past this phase before the warp acts.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t phase, int where, volatile int* abort) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait_abortable(bar, phase, where, abort);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) ok = mbar_try_wait(bar, phase) ? 1 : 0;
+  return __all_sync(0xffffffffu, ok) != 0;
+}
+
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
                                             int c2) {
   asm volatile(

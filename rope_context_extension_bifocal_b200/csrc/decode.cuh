@@ -11,10 +11,11 @@
 // is read once from HBM and never rewritten. G follows the current length L, so when
 // L crosses a multiple of w_pretrained every long-range key is re-phased at once.
 //
-// Work split: CTA = (key range, up to 8 kv heads); a producer warp streams 16-key stages
-// (K and V, every head, both 64-element halves of D) through a 3-deep mbarrier ring, and
-// two consumer warps per kv head each take one 8-key n-tile of every stage, keeping their
-// own online softmax (each warp is a split of its own for the combine). QK^T of the
+// Work split: CTA = (key range, up to 4 kv heads). A TMA warp streams 16-key stages
+// (K and V, every head, both 64-element halves of D) through a 5-deep mbarrier ring, two
+// table warps build each stage's correction cos/sin table; two consumer warps per kv head each take
+// one 8-key n-tile of every stage, keeping their own online softmax (each warp is a split
+// of its own for the combine). QK^T of the
 // g = hq/hkv query rows runs on mma.sync m16n8k16 (rows in M); PV runs transposed,
 // O^T = V^T P^T on m16n8k8, so the query rows sit in N and the accumulator is D x 8.
 // QK^T operands are fp16 (rotated query, corrected or converted cached key), PV is bf16.
@@ -25,8 +26,8 @@ namespace bf {
 
 namespace dec {
 constexpr int KB = 16;      // keys per stage
-constexpr int NST = 2;      // stages in flight (2 x 64 KB per SM is ample for HBM latency)
-constexpr int HPC = 8;      // kv heads per CTA (max)
+constexpr int NST = 5;      // stages in the ring (4 in flight while one is consumed)
+constexpr int HPC = 4;      // kv heads per CTA (max)
 constexpr int MAX_G = 8;    // query heads per kv head (max)
 }  // namespace dec
 
@@ -34,8 +35,8 @@ struct DecodeArgs {
   CUtensorMap kmap;  // cache K viewed as (d_lo 64, d_hi D/64, head hkv, key cap), box (64,1,1,KB)
   CUtensorMap vmap;
   const __nv_bfloat16* q;  // [hq, D] raw
-  float* part_o;           // [n_split, hq, D] unnormalised
-  float* part_ml;          // [n_split, hq, 2]: running max (log2 domain), sum
+  float* part_o;           // [2 * n_split, hq, D] unnormalised
+  float* part_ml;          // [2 * n_split, hq, 2]: running max (log2 domain), sum
   int L, hq, hkv, w0, G, mode, bifocal;
   int split_len, n_split;
   float scale_log2;
@@ -50,7 +51,7 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
 }
 
 template <int D>
-__global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
   using namespace dec;
   constexpr int P = D / 2;
   constexpr int HALVES = D / 64;
@@ -58,15 +59,15 @@ __global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_ker
   constexpr int KCP = KC / 2;      // k-chunks holding the first element of each pair
   constexpr int MT = D / 16;       // m-tiles of O^T (16 d-values each)
   constexpr uint32_t HEAD_TILE = KB * 128;                 // one head, one half: KB rows x 128 B
-  constexpr uint32_t STAGE_KV = HPC * HALVES * HEAD_TILE;  // all heads, all halves
+  constexpr uint32_t STAGE_KV = HPC * HALVES * HEAD_TILE;  // all heads, all halves (K or V)
   constexpr int CS_STRIDE = P * 8 + 64;  // bytes per key row of the cos/sin table (pad: rows 16 banks apart)
+  constexpr uint32_t STAGE_CS = KB * CS_STRIDE;
 
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sK = smem;                       // [NST][HPC][HALVES][KB][128 B]
   uint8_t* sV = sK + NST * STAGE_KV;        // same
-  uint8_t* sCS = sV + NST * STAGE_KV;       // [2][KB][CS_STRIDE]
-  uint4* sQA = reinterpret_cast<uint4*>(sCS + 2 * KB * CS_STRIDE);  // [HPC][KC][32 lanes] query fragments
-  uint64_t* full = reinterpret_cast<uint64_t*>(sQA + HPC * KC * 32);
+  uint8_t* sCS = sV + NST * STAGE_KV;       // [NST][KB][CS_STRIDE]: correction cos/sin per stage
+  uint64_t* full = reinterpret_cast<uint64_t*>(sCS + NST * STAGE_CS);
   uint64_t* empty = full + NST;
   __shared__ int s_abort;  // set when a bounded wait expires: later waits return at once
 
@@ -84,7 +85,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_ker
   if (threadIdx.x == 0) {
     s_abort = 0;
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + 32);  // producer's expect_tx + one arrive per producer lane (cos/sin written)
       mbar_init(&empty[s], nconsumers);
     }
     fence_barrier_init();
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_ker
   __syncthreads();
 
   if (warp == 2 * HPC) {
-    // producer: one elected lane streams the stages
+    // ---------------- TMA warp: one elected lane streams K/V stages
     if (lane == 0) {
       prefetch_tensormap(&a.kmap);
       prefetch_tensormap(&a.vmap);
@@ -100,8 +101,8 @@ __global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_ker
       for (int s = 0; s < nstage; ++s) {
         const int st = s % NST;
         if (s >= NST && !mbar_wait_abortable(&empty[st], ((s / NST) - 1) & 1, 1, &s_abort)) break;
-        mbar_arrive_expect_tx(&full[st], bytes);
         const int j0 = jbeg + s * KB;
+        mbar_arrive_expect_tx(&full[st], bytes);
         for (int hh = 0; hh < nheads; ++hh)
           for (int hf = 0; hf < HALVES; ++hf) {
             const uint32_t off = st * STAGE_KV + (hh * HALVES + hf) * HEAD_TILE;
@@ -112,6 +113,64 @@ __global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_ker
     }
     return;
   }
+  if (warp > 2 * HPC) {
+    // ---------------- table warps (two, alternating stages): correction cos/sin per (key, pair).
+    // Each lane runs 4 chains (pairs lane and lane + 32, keys 0-7 and 8-15 of the stage): an
+    // exact angle at the chain's first key, then per-key steps: frequency interpolation adds
+    // omega_corr; position aliasing adds -omega unless the next key starts a group of G.
+    const int cw = warp - 2 * HPC - 1;  // 0 or 1
+    float fi_c[2], fi_s[2], pa_c[2], pa_s[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int pr = lane + 32 * e;
+      fi_c[e] = pa_c[e] = 1.f;
+      fi_s[e] = pa_s[e] = 0.f;
+      if (pr < P) {
+        angle_cos_sin(a.omega_corr[pr], fi_c[e], fi_s[e]);
+        angle_cos_sin(-a.omega[pr], pa_c[e], pa_s[e]);
+      }
+    }
+    for (int s = cw; s < nstage; s += 2) {
+      const int st = s % NST;
+      if (s >= NST && !__all_sync(0xffffffffu, mbar_wait_abortable(&empty[st], ((s / NST) - 1) & 1, 3, &s_abort)))
+        break;
+      const int j0 = jbeg + s * KB;
+      if (j0 < local_from) {  // some key of this stage is long-range
+        uint8_t* cs = sCS + st * STAGE_CS;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int pr = lane + 32 * e;
+          if (pr >= P) continue;
+          float c[2], sn[2];
+#pragma unroll
+          for (int hk = 0; hk < 2; ++hk) {
+            const int jc = j0 + 8 * hk;
+            const double ang0 = (a.mode == 0) ? static_cast<double>(jc) * a.omega_corr[pr]
+                                              : static_cast<double>(jc / a.G - jc) * a.omega[pr];
+            angle_cos_sin(ang0, c[hk], sn[hk]);
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+            for (int hk = 0; hk < 2; ++hk) {
+              *reinterpret_cast<float2*>(cs + (8 * hk + kk) * CS_STRIDE + pr * 8) = make_float2(c[hk], sn[hk]);
+              float dc = fi_c[e], ds = fi_s[e];
+              if (a.mode != 0) {
+                const bool stay = ((j0 + 8 * hk + kk + 1) % a.G) == 0;
+                dc = stay ? 1.f : pa_c[e];
+                ds = stay ? 0.f : pa_s[e];
+              }
+              const float nc = c[hk] * dc - sn[hk] * ds;
+              sn[hk] = sn[hk] * dc + c[hk] * ds;
+              c[hk] = nc;
+            }
+          }
+        }
+      }
+      mbar_arrive(&full[st]);  // every lane: its table entries are written
+    }
+    return;
+  }
   if (warp >= nconsumers) return;  // fewer kv heads than warp pairs in this CTA
 
   // ---------------- consumers: warp pair (2h, 2h+1) handles kv head head0 + h ----------------
@@ -119,18 +178,15 @@ __global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_ker
   const int kvh = head0 + hl;
   const int g8 = lane >> 2, t4 = lane & 3;
 
-  // Query fragments (rows 0..g-1 = the g query heads of this kv head) under both RoPE
-  // forms, fp16, in the m16n8k16 A layout: per k-chunk pair (kc, kc + KC/2) a lane holds
-  // {orig a0, orig a2} of chunk kc and chunk kc + KC/2 ... stored as two uint4 per kc:
-  // sQA[hl][kc][lane] = {o(kc).a0, o(kc).a2, l(kc).a0, l(kc).a2}, kc < KC (rows 8..15 are zero).
-  if (nt == 0) {
+  // query fragments (rows 0..g-1 = the g query heads of this kv head) under both RoPE forms,
+  // fp16, in the m16n8k16 A layout: qa_*[kc] = {a0, a2} of k-chunk kc (rows 8..15 are zero)
+  uint32_t qa_o[KC][2], qa_l[KC][2];
+  {
     const bool row_ok = g8 < g;
     const __nv_bfloat16* qrow = a.q + static_cast<long long>(kvh * g + (row_ok ? g8 : 0)) * D;
     const double pl = (a.mode == 0) ? static_cast<double>(p) : static_cast<double>(p / a.G);
-    uint4* dst = sQA + hl * KC * 32;
 #pragma unroll
-    for (int kc = 0; kc < KCP; ++kc) {
-      uint32_t fo[2][2], fl[2][2];  // [first/second element of the pair][sub]
+    for (int kc = 0; kc < KCP; ++kc)
 #pragma unroll
       for (int sub = 0; sub < 2; ++sub) {
         const int d = 16 * kc + 8 * sub + 2 * t4;  // pair indices d, d + 1
@@ -153,53 +209,32 @@ __global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_ker
           xl[e] = x * c - y * sn;
           yl[e] = y * c + x * sn;
         }
-        fo[0][sub] = pack_f16x2(xo[0], xo[1]);
-        fo[1][sub] = pack_f16x2(yo[0], yo[1]);
-        fl[0][sub] = pack_f16x2(xl[0], xl[1]);
-        fl[1][sub] = pack_f16x2(yl[0], yl[1]);
+        qa_o[kc][sub] = pack_f16x2(xo[0], xo[1]);
+        qa_o[kc + KCP][sub] = pack_f16x2(yo[0], yo[1]);
+        qa_l[kc][sub] = pack_f16x2(xl[0], xl[1]);
+        qa_l[kc + KCP][sub] = pack_f16x2(yl[0], yl[1]);
       }
-      dst[(2 * kc) * 32 + lane] = make_uint4(fo[0][0], fo[0][1], fl[0][0], fl[0][1]);      // chunk kc
-      dst[(2 * kc + 1) * 32 + lane] = make_uint4(fo[1][0], fo[1][1], fl[1][0], fl[1][1]);  // chunk kc + KC/2
-    }
   }
-  const uint4* qfrag = sQA + hl * KC * 32;
 
   // O^T [D x 8 query rows]: o[mt][0..1] = d = 16mt + g8, rows 2t4, 2t4+1; o[mt][2..3] = d + 8
   float o[MT][4];
 #pragma unroll
   for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m_r = -INFINITY, l_r = 0.f;  // softmax state of query row g8 (S layout)
-  const int nthr = nconsumers * 32;
-  const int tid = threadIdx.x;
 
   for (int s = 0; s < nstage; ++s) {
     const int st = s % NST;
     const int j0 = jbeg + s * KB;
-    const bool any_long = j0 < local_from;
     const int jt = j0 + nt * 8;  // first key of this warp's n-tile
     const bool tile_long = jt < local_from;
     const bool tile_local = jt + 7 >= local_from;
-    // cooperative cos/sin table of the correction rotation for this stage's keys
-    uint8_t* cs = sCS + (s & 1) * KB * CS_STRIDE;
-    if (any_long) {
-      for (int idx = tid; idx < KB * P; idx += nthr) {
-        const int kk = idx / P, pr = idx % P;
-        const int j = j0 + kk;
-        const double ang = (a.mode == 0) ? static_cast<double>(j) * a.omega_corr[pr]
-                                         : static_cast<double>(j / a.G - j) * a.omega[pr];
-        float c, sn;
-        angle_cos_sin(ang, c, sn);
-        *reinterpret_cast<float2*>(cs + kk * CS_STRIDE + pr * 8) = make_float2(c, sn);
-      }
-    }
-    asm volatile("bar.sync 1, %0;\n" ::"r"(nthr));  // also publishes the query fragments
-    // after an expired wait every warp still takes part in the barriers but computes nothing
-    if (!mbar_wait_abortable(&full[st], (s / NST) & 1, 2, &s_abort)) {
+    // warp-uniform result: the ldmatrix / mma.sync below are warp-collective
+    if (!__all_sync(0xffffffffu, mbar_wait_abortable(&full[st], (s / NST) & 1, 2, &s_abort))) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
       continue;
     }
-
+    const uint8_t* cs = sCS + st * STAGE_CS;
     const uint32_t kbase = smem_u32(sK + st * STAGE_KV + hl * HALVES * HEAD_TILE);
     const uint32_t vbase = smem_u32(sV + st * STAGE_KV + hl * HALVES * HEAD_TILE);
     float so[4] = {0.f, 0.f, 0.f, 0.f}, sl[4] = {0.f, 0.f, 0.f, 0.f};
@@ -211,10 +246,9 @@ __global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_ker
       const int e_lo = 16 * kc + 8 * ((lane >> 3) & 1) + ((lane >> 4) ? P : 0);
       uint32_t r[4];
       ldmatrix_x4(r, kbase + (e_lo / 64) * HEAD_TILE + sw128(krow, (e_lo % 64) / 8));
-      const uint4 qf0 = qfrag[(2 * kc) * 32 + lane], qf1 = qfrag[(2 * kc + 1) * 32 + lane];
       if (tile_local) {
-        uint32_t a0[4] = {qf0.x, 0u, qf0.y, 0u};
-        uint32_t a1[4] = {qf1.x, 0u, qf1.y, 0u};
+        uint32_t a0[4] = {qa_o[kc][0], 0u, qa_o[kc][1], 0u};
+        uint32_t a1[4] = {qa_o[kc + KCP][0], 0u, qa_o[kc + KCP][1], 0u};
         mma_f16_16816(so, a0, bf16x2_to_f16x2(r[0]), bf16x2_to_f16x2(r[1]));
         mma_f16_16816(so, a1, bf16x2_to_f16x2(r[2]), bf16x2_to_f16x2(r[3]));
       }
@@ -228,8 +262,8 @@ __global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_ker
         const uint32_t ry0 = pack_f16x2(y0.x * c01.x + x0.x * c01.y, y0.y * c01.z + x0.y * c01.w);
         const uint32_t rx1 = pack_f16x2(x1.x * c89.x - y1.x * c89.y, x1.y * c89.z - y1.y * c89.w);
         const uint32_t ry1 = pack_f16x2(y1.x * c89.x + x1.x * c89.y, y1.y * c89.z + x1.y * c89.w);
-        uint32_t a0[4] = {qf0.z, 0u, qf0.w, 0u};
-        uint32_t a1[4] = {qf1.z, 0u, qf1.w, 0u};
+        uint32_t a0[4] = {qa_l[kc][0], 0u, qa_l[kc][1], 0u};
+        uint32_t a1[4] = {qa_l[kc + KCP][0], 0u, qa_l[kc + KCP][1], 0u};
         mma_f16_16816(sl, a0, rx0, rx1);
         mma_f16_16816(sl, a1, ry0, ry1);
       }
@@ -304,13 +338,12 @@ __global__ void __launch_bounds__((2 * dec::HPC + 1) * 32, 1) decode_partial_ker
 
 template <int D>
 constexpr int decode_smem_bytes() {
-  return 2 * dec::NST * dec::HPC * (D / 64) * dec::KB * 128 + 2 * dec::KB * (D / 2 * 8 + 64) +
-         dec::HPC * (D / 16) * 32 * 16 + 2 * dec::NST * 8;
+  return 2 * dec::NST * dec::HPC * (D / 64) * dec::KB * 128 + dec::NST * dec::KB * (D / 2 * 8 + 64) + 2 * dec::NST * 8;
 }
 
 template <int D>
 constexpr int decode_threads() {
-  return (2 * dec::HPC + 1) * 32;
+  return (2 * dec::HPC + 3) * 32;  // consumers, TMA warp, two table warps
 }
 
 // Log-sum-exp merge of the split partials: one CTA per query head, one thread per d.

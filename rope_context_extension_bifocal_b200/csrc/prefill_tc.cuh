@@ -9,10 +9,12 @@
 // so both GEMMs read only their B operand (a K or V tile) from shared memory. K and V
 // tiles (128 keys x 128 d) arrive by TMA into a ring of 32 KB slots.
 //
-// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (one thread), warps 2..5 =
-// softmax (thread = query row; warp w reads TMEM lanes 32*(w%4)..). Per key tile the
-// MMA warp issues S = Q K^T into the free S buffer while the softmax works on the other
-// one, then O += P V once the softmax has published P.
+// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (one thread), warps 2..9 =
+// softmax. A softmax thread owns one query row and one half of the 128 key columns (warp w
+// reads TMEM lanes 32*(w%4).., warps 2-5 the left half, 6-9 the right half); the two halves
+// of a row exchange their maxima through shared memory. Per key tile the MMA warp issues
+// S = Q K^T into the free S buffer while the softmax works on the other one, then
+// O += P V once the softmax has published P.
 //
 // Bifocal structure (ai-feeds summary of Jet-Long, 方法 key modules 1 and 3): a key tile
 // whose pairs all lie inside the local window (i - j < w0) is scored with the original
@@ -32,7 +34,7 @@ constexpr int D = 128;
 constexpr int NSLOT = 6;
 constexpr uint32_t SLOT_BYTES = 32768;  // one K or V tile: two 128-row x 128-byte swizzled halves
 constexpr uint32_t HALF_BYTES = 16384;
-constexpr int NTHREADS = 192;  // 6 warps
+constexpr int NTHREADS = 320;  // 10 warps: TMA, MMA, 8 softmax (two per TMEM lane quadrant)
 constexpr uint32_t COL_QO = 0, COL_QL = 64, COL_S = 128, COL_O = 384, NCOLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.f;  // log2 units: O is rescaled only when the row max grows by more
 
@@ -146,6 +148,7 @@ __global__ void __launch_bounds__(tc::NTHREADS, 1) attn_tc_kernel(const __grid_c
   __shared__ uint64_t full[NSLOT], empty[NSLOT], s_full[2], p_ready[2], o_done, q_ready, mma_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int s_abort;
+  __shared__ float red[2][2][BM];  // [visit parity][column half][row]: row maxima, then row sums
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = (a.L + BM - 1) / BM;
@@ -166,10 +169,10 @@ __global__ void __launch_bounds__(tc::NTHREADS, 1) attn_tc_kernel(const __grid_c
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_ready[i], 4);
+      mbar_init(&p_ready[i], 8);
     }
     mbar_init(&o_done, 1);
-    mbar_init(&q_ready, 4);
+    mbar_init(&q_ready, 8);
     mbar_init(&mma_drain, 1);
     fence_barrier_init();
   }
@@ -284,29 +287,31 @@ __global__ void __launch_bounds__(tc::NTHREADS, 1) attn_tc_kernel(const __grid_c
       mbar_wait(&mma_drain, 0, 26);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps 2..5
-    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
-    const int r = quad * 32 + lane;  // row within the tile
-    const int i = i0 + r;            // query row
+    // ------------------------------------------------------------ softmax warps 2..9
+    const int quad = warp & 3;          // TMEM lane quadrant this warp may access
+    const int half = (warp - 2) >> 2;   // which 64 of the 128 key columns
+    const int r = quad * 32 + lane;     // row within the tile
+    const int i = i0 + r;               // query row
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    // Q (both RoPE forms) into TMEM: lane = row, 64 columns of fp16 pairs each
+    const uint32_t bar_id = 1 + quad;   // named barrier of the two warps sharing these rows
+    // Q (both RoPE forms) into TMEM: lane = row, 64 columns of fp16 pairs each; each half
+    // of the row's threads writes 32 columns of each form
     {
       const long long qrow = ((static_cast<long long>(b) * a.hq + h) * a.L + i) * D;
       for (int f = 0; f < (BIFOCAL ? 2 : 1); ++f) {
         const __half* src = (f == 0 ? a.Qo : a.Ql) + qrow;
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          uint32_t reg[32];
+        const int c0 = 32 * half;
+        uint32_t reg[32];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            uint4 x = make_uint4(0u, 0u, 0u, 0u);
-            if (i < a.L) x = reinterpret_cast<const uint4*>(src)[c0 / 4 + u];
-            reg[4 * u + 0] = x.x;
-            reg[4 * u + 1] = x.y;
-            reg[4 * u + 2] = x.z;
-            reg[4 * u + 3] = x.w;
-          }
-          tmem_st32(lane_addr + (f == 0 ? COL_QO : COL_QL) + c0, reg);
+        for (int u = 0; u < 8; ++u) {
+          uint4 x = make_uint4(0u, 0u, 0u, 0u);
+          if (i < a.L) x = reinterpret_cast<const uint4*>(src)[c0 / 4 + u];
+          reg[4 * u + 0] = x.x;
+          reg[4 * u + 1] = x.y;
+          reg[4 * u + 2] = x.z;
+          reg[4 * u + 3] = x.w;
         }
+        tmem_st32(lane_addr + (f == 0 ? COL_QO : COL_QL) + c0, reg);
       }
       wait_st();
       fence_before();
@@ -314,101 +319,118 @@ __global__ void __launch_bounds__(tc::NTHREADS, 1) attn_tc_kernel(const __grid_c
       if (lane == 0) mbar_arrive(&q_ready);
     }
 
-    float m_ref = -INFINITY, l_sum = 0.f;
+    // After an expired wait (ok == false, warp-uniform) a warp does no more work but still
+    // passes every named barrier its partner warp passes, so the pair cannot deadlock.
+    float m_ref = -INFINITY, l_half = 0.f;
     int v = 0;
     bool ok = true;
-    for (int t = 0; t < n_kt && ok; ++t) {
+    for (int t = 0; t < n_kt; ++t) {
       int kinds[2];
       const int nv = tile_visits<BIFOCAL>(i0, t, a.w0, kinds);
       const int j0 = t * BN;
-      for (int vi = 0; vi < nv && ok; ++vi, ++v) {
+      for (int vi = 0; vi < nv; ++vi, ++v) {
         const int kind = kinds[vi];
-        if (!mbar_wait_abortable(&s_full[v & 1], (v >> 1) & 1, 30, &s_abort)) {
-          ok = false;
-          break;
-        }
-        fence_after();
+        // every lane waits; the result is made warp-uniform because the TMEM accesses
+        // below are warp-collective (.sync.aligned)
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_abortable(&s_full[v & 1], (v >> 1) & 1, 30, &s_abort));
         const uint32_t s_addr = lane_addr + COL_S + (v & 1) * 128;
-        float s[128];
-#pragma unroll
-        for (int c = 0; c < 128; c += 32) tmem_ld32(s_addr + c, s + c);
-        wait_ld();
-        // scale, mask, row max
-        const bool masked = kind != LONG_FULL && (kind != ORIG_FULL || j0 + BN - 1 > i0);
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float x = s[c] * a.scale_log2;
-          if (masked) {
-            const int d = i - (j0 + c);
-            bool keep;
-            if (kind == ORIG_FULL)
-              keep = d >= 0;
-            else if (kind == ORIG_LOCAL)
-              keep = d >= 0 && d < a.w0;
-            else
-              keep = d >= a.w0;
-            x = keep ? x : -INFINITY;
-          }
-          s[c] = x;
-          mx = fmaxf(mx, x);
-        }
-        // lazy rescale: keep the old reference unless the max grew by more than the threshold
-        float alpha = 1.f;
-        bool rescale = false;
-        if (mx > m_ref + RESCALE_THRESHOLD || (m_ref == -INFINITY && mx > -INFINITY)) {
-          alpha = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mx);
-          rescale = m_ref != -INFINITY;
-          m_ref = mx;
-        }
-        const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float rs = 0.f;
-        uint32_t pk[64];
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float p0 = fast_exp2(s[c] - ref), p1 = fast_exp2(s[c + 1] - ref);
-          rs += p0 + p1;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-        }
-        l_sum = l_sum * alpha + rs;
-        tmem_st32(s_addr, pk);
-        tmem_st32(s_addr + 32, pk + 32);
-        // O must hold PV(v-1) before it is rescaled and before PV(v) adds to it
-        if (v >= 1) {
-          if (!mbar_wait_abortable(&o_done, (v - 1) & 1, 31, &s_abort)) {
-            ok = false;
-            break;
-          }
+        float s[64];
+        float mh = -INFINITY;
+        if (ok) {
           fence_after();
-          if (rescale) {
-            const uint32_t o_addr = lane_addr + COL_O;
-#pragma unroll 1
-            for (int c = 0; c < 128; c += 32) {
-              float ov[32];
-              tmem_ld32(o_addr + c, ov);
-              wait_ld();
-              uint32_t ou[32];
+          tmem_ld32(s_addr + 64 * half, s);
+          tmem_ld32(s_addr + 64 * half + 32, s + 32);
+          wait_ld();
+          // mask (only on visits that need one)
+          const bool masked = kind != LONG_FULL && (kind != ORIG_FULL || j0 + BN - 1 > i0);
+          if (masked) {
+            const int d0 = i - j0 - 64 * half;  // i - j for this thread's first column
+            const int lo = (kind == LONG_ONLY) ? a.w0 : 0;            // keep lo <= i - j
+            const int hi = (kind == ORIG_LOCAL) ? a.w0 : 0x7fffffff;  //      and i - j < hi
 #pragma unroll
-              for (int u = 0; u < 32; ++u) ou[u] = __float_as_uint(ov[u] * alpha);
-              tmem_st32(o_addr + c, ou);
+            for (int c = 0; c < 64; ++c) {
+              const int d = d0 - c;
+              s[c] = (d >= lo && d < hi) ? s[c] : -INFINITY;
             }
           }
+          // raw max of this half with independent accumulators
+          float m8[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) m8[u] = s[u];
+#pragma unroll
+          for (int c = 8; c < 64; c += 8)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) m8[u] = fmaxf(m8[u], s[c + u]);
+          mh = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         }
-        wait_st();
-        fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_ready[v & 1]);
+        // the row max with the other half
+        red[v & 1][half][r] = mh;
+        asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+        mh = fmaxf(mh, red[v & 1][half ^ 1][r]);
+        if (ok) {
+          const float mx = mh * a.scale_log2;  // scale > 0: max commutes with it
+          // lazy rescale (both halves take the same decision): a row keeps its reference
+          // unless its max grew by more than the threshold
+          float alpha = 1.f;
+          bool grow = false;
+          if (mx > m_ref + RESCALE_THRESHOLD || (m_ref == -INFINITY && mx > -INFINITY)) {
+            alpha = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mx);
+            grow = m_ref != -INFINITY;  // O already holds this row's earlier terms
+            m_ref = mx;
+          }
+          const float neg_ref = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          const float sc = a.scale_log2;
+          float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float p0 = fast_exp2(fmaf(s[c], sc, neg_ref)), p1 = fast_exp2(fmaf(s[c + 1], sc, neg_ref));
+            r8[(c >> 1) & 7] += p0 + p1;
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+          }
+          const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+          l_half = l_half * alpha + rs;
+          tmem_st32(s_addr + 32 * half, pk);  // P (bf16 pairs) over the first 64 columns of the S buffer
+          // O must hold PV(v-1) before it is rescaled and before PV(v) adds to it
+          if (v >= 1) ok = __all_sync(0xffffffffu, mbar_wait_abortable(&o_done, (v - 1) & 1, 31, &s_abort));
+          if (ok && v >= 1) {
+            fence_after();
+            // warp-uniform: rescale this half of O if any row of the warp needs it (others scale by 1)
+            if (__any_sync(0xffffffffu, grow)) {
+              const float f = grow ? alpha : 1.f;
+              const uint32_t o_addr = lane_addr + COL_O + 64 * half;
+#pragma unroll 1
+              for (int c = 0; c < 64; c += 32) {
+                float ov[32];
+                tmem_ld32(o_addr + c, ov);
+                wait_ld();
+                uint32_t ou[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) ou[u] = __float_as_uint(ov[u] * f);
+                tmem_st32(o_addr + c, ou);
+              }
+            }
+          }
+          wait_st();
+          fence_before();
+          __syncwarp();
+          if (ok && lane == 0) mbar_arrive(&p_ready[v & 1]);
+        }
       }
     }
-    // epilogue: O / l -> bf16, LSE
-    if (ok && v >= 1 && mbar_wait_abortable(&o_done, (v - 1) & 1, 32, &s_abort)) {
+    // epilogue: row sum of both halves, O / l -> bf16 (each half its 64 columns), LSE
+    const bool fin = ok && v >= 1 && __all_sync(0xffffffffu, mbar_wait_abortable(&o_done, (v - 1) & 1, 32, &s_abort));
+    red[0][half][r] = l_half;
+    asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+    const float l_sum = l_half + red[0][half ^ 1][r];
+    if (fin) {
       fence_after();
       const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      __nv_bfloat16* orow = a.out + ((static_cast<long long>(b) * a.L + i) * a.hq + h) * D;
+      __nv_bfloat16* orow = a.out + ((static_cast<long long>(b) * a.L + i) * a.hq + h) * D + 64 * half;
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         float ov[32];
-        tmem_ld32(lane_addr + COL_O + c, ov);
+        tmem_ld32(lane_addr + COL_O + 64 * half + c, ov);
         wait_ld();
         if (i < a.L) {
 #pragma unroll
@@ -422,7 +444,7 @@ __global__ void __launch_bounds__(tc::NTHREADS, 1) attn_tc_kernel(const __grid_c
           }
         }
       }
-      if (a.lse && i < a.L)
+      if (half == 0 && a.lse && i < a.L)
         a.lse[(static_cast<long long>(b) * a.hq + h) * a.L + i] = (m_ref + __log2f(l_sum)) * 0.69314718055994530942f;
     }
   }

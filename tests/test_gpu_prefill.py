@@ -94,11 +94,13 @@ def test_plain_comparator_matches_oracle():
 
 @pytest.mark.parametrize("mode", [si.FREQ_INTERP, si.POS_ALIAS])
 def test_forced_bifocal_equals_shortcut_when_g1(mode):
-    # G == 1: both branches coincide; the two-branch kernel must give the plain kernel's bits
+    # G == 1: both branches coincide, so the two-branch kernel must reproduce the plain kernel up to
+    # fp32 summation order (band-edge tiles are accumulated in two visits instead of one)
     q, k, v = si.random_qkv(9, 1, 500, 4, 2, 128, "bf16")
     a, la, _, _ = run_prefill(q, k, v, 64, 512, 1e6, mode)
     b, lb, _, _ = run_prefill(q, k, v, 64, 512, 1e6, mode, flags=bfl.FLAG_FORCE_BIFOCAL)
-    assert torch.equal(a, b) and torch.equal(la, lb)
+    assert (a.float() - b.float()).abs().max().item() <= 2.0 ** -7 * max(1.0, a.float().abs().max().item())
+    assert (la - lb).abs().max().item() <= 1e-5
 
 
 def test_kv_cache_output():
