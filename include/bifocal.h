@@ -155,6 +155,24 @@ BF_API bf_status_t bifocal_decode(const void* q, const void* k_new, const void* 
                            int32_t cap, int32_t L, const bf_params_t* p, void* out, float* lse, void* workspace,
                            size_t ws_bytes, void* stream);
 
+/* bifocal_decode without a caller workspace, for callers that cannot allocate device memory
+ * themselves: for example a plug-in hosted by a runtime that owns and pre-plans all device
+ * memory, or a latency-critical loop that may not call cudaMalloc (which synchronises the
+ * device). There is no counterpart in the paper; this is a deployment convenience.
+ * The split-KV partials live in a static device array of BIFOCAL_NOALLOC_SCRATCH_BYTES
+ * (16 MiB) that every GPU loading the library holds until the process exits. A call needs
+ * bifocal_decode_workspace_size(L, p) bytes of it (10.7 MB for 32 query heads of 128);
+ * larger problems are rejected with BF_ERR_WORKSPACE before any launch.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents: nothing in it needs
+ * to start at zero, but calls that overlap on the GPU (other streams, other threads) race
+ * on it and must be serialised by the caller. Arguments and errors as bifocal_decode. */
+#define BIFOCAL_NOALLOC_SCRATCH_BYTES (16u << 20)
+BF_API bf_status_t bifocal_decode_noalloc(const void* q, const void* k_new, const void* v_new, void* kcache,
+                                          void* vcache, int32_t cap, int32_t L, const bf_params_t* p, void* out,
+                                          float* lse, void* stream);
+
 /* Plain-RoPE decode step (comparator): same arguments; every cached key is used as stored. */
 BF_API bf_status_t rope_causal_decode(const void* q, const void* k_new, const void* v_new, void* kcache, void* vcache,
                                int32_t cap, int32_t L, const bf_params_t* p, void* out, float* lse,

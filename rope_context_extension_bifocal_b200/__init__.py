@@ -15,7 +15,7 @@ from typing import Optional, Tuple
 
 __all__ = [
     "BifocalError", "FREQ_INTERP", "POS_ALIAS", "FLAG_FORCE_BIFOCAL", "FLAG_MMA_SYNC", "Params", "lib", "lib_path",
-    "bifocal_factor", "bifocal_prefill", "bifocal_prefill_rope", "bifocal_prefill_attention", "rope_causal_prefill", "bifocal_decode", "rope_causal_decode",
+    "bifocal_factor", "bifocal_prefill", "bifocal_prefill_rope", "bifocal_prefill_attention", "rope_causal_prefill", "bifocal_decode", "bifocal_decode_noalloc", "rope_causal_decode",
     "prefill_workspace_size", "decode_workspace_size", "last_device_error", "build_info",
 ]
 
@@ -75,6 +75,8 @@ def _lib() -> ctypes.CDLL:
         dec = [vp, vp, vp, vp, vp, i32, i32, pp, vp, vp, vp, sz, vp]
         for name in ("bifocal_decode", "rope_causal_decode"):
             getattr(L, name).argtypes, getattr(L, name).restype = dec, i32
+        L.bifocal_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, pp, vp, vp, vp]
+        L.bifocal_decode_noalloc.restype = i32
         L.bifocal_status_string.argtypes, L.bifocal_status_string.restype = [i32], ctypes.c_char_p
         L.bifocal_last_device_error.argtypes, L.bifocal_last_device_error.restype = [vp], i32
         L.bifocal_build_info.argtypes, L.bifocal_build_info.restype = [], ctypes.c_char_p
@@ -224,6 +226,27 @@ def bifocal_decode(q, k_new, v_new, kcache, vcache, L: int, *, w0: int, w_pretra
     kcache / vcache [cap, Hkv, D] bf16 (original-RoPE keys); row L-1 is written. Returns (out, lse)."""
     p = make_params(q.shape[0], k_new.shape[0], q.shape[1], w0, w_pretrained, theta, mode, scale, flags)
     return _decode("bifocal_decode", q, k_new, v_new, kcache, vcache, L, p, want_lse, out, workspace, stream)
+
+
+def bifocal_decode_noalloc(q, k_new, v_new, kcache, vcache, L: int, *, w0: int, w_pretrained: int, theta: float,
+                           mode: str = FREQ_INTERP, scale: Optional[float] = None, flags: int = 0,
+                           want_lse: bool = True, out=None, lse=None, stream=None):
+    """bifocal_decode with the library's static scratch instead of a workspace.
+
+    For callers that cannot allocate device memory themselves. Pass preallocated `out`
+    (and `lse`) to keep the call itself free of allocations; calls that overlap on the GPU
+    share the scratch and race (see include/bifocal.h)."""
+    import torch
+    hq, D = q.shape
+    p = make_params(hq, k_new.shape[0], D, w0, w_pretrained, theta, mode, scale, flags)
+    out = torch.empty(hq, D, dtype=torch.bfloat16, device=q.device) if out is None else out
+    if want_lse and lse is None:
+        lse = torch.empty(hq, dtype=torch.float32, device=q.device)
+    st = _lib().bifocal_decode_noalloc(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(kcache), _ptr(vcache),
+                                       kcache.shape[0], int(L), ctypes.byref(p), _ptr(out),
+                                       _ptr(lse if want_lse else None), _stream(stream))
+    _check(st, "bifocal_decode_noalloc")
+    return out, (lse if want_lse else None)
 
 
 def rope_causal_decode(q, k_new, v_new, kcache, vcache, L: int, *, theta: float, scale: Optional[float] = None,

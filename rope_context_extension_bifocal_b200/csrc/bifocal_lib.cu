@@ -409,6 +409,29 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
   return cudaGetLastError() == cudaSuccess ? BF_OK : BF_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ allocation-free decode
+// Static scratch for bifocal_decode_noalloc: holds the split-KV partials. Every call shares
+// it; overlapping calls race (documented in the header).
+__device__ __align__(256) uint8_t g_noalloc_scratch[BIFOCAL_NOALLOC_SCRATCH_BYTES];
+
+// Host code cannot use the array's name as a device address: look the address up once per
+// device, with that device current.
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+void* noalloc_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -458,6 +481,19 @@ bf_status_t bifocal_decode(const void* q, const void* k_new, const void* v_new, 
                            int32_t cap, int32_t L, const bf_params_t* p, void* out, float* lse, void* workspace,
                            size_t ws_bytes, void* stream) {
   return decode_impl(true, q, k_new, v_new, kcache, vcache, cap, L, p, out, lse, workspace, ws_bytes, stream);
+}
+
+bf_status_t bifocal_decode_noalloc(const void* q, const void* k_new, const void* v_new, void* kcache, void* vcache,
+                                   int32_t cap, int32_t L, const bf_params_t* p, void* out, float* lse, void* stream) {
+  bf_status_t s = check_params(p, true);
+  if (s != BF_OK) return s;
+  if (L < 1 || cap < L) return BF_ERR_INVALID;
+  const size_t need = decode_layout(L, p).total;
+  if (need > BIFOCAL_NOALLOC_SCRATCH_BYTES) return BF_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch_ptr();
+  if (!scratch) return BF_ERR_CUDA;
+  return decode_impl(true, q, k_new, v_new, kcache, vcache, cap, L, p, out, lse, scratch,
+                     BIFOCAL_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 bf_status_t rope_causal_decode(const void* q, const void* k_new, const void* v_new, void* kcache, void* vcache,
