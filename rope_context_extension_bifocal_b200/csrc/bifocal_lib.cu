@@ -13,6 +13,7 @@
 #include "decode.cuh"
 #include "prefill_mma.cuh"
 #include "prefill_tc.cuh"
+#include "prefill_tc2.cuh"
 #include "rope_prepass.cuh"
 
 namespace {
@@ -261,8 +262,34 @@ bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtyp
   aa.w0 = plan.bif ? p->w0 : L;
   aa.scale_log2 = scale_log2(p);
   cudaError_t e;
-  if (D == 128 && !(p->flags & BF_FLAG_MMA_SYNC)) {
-    // tcgen05 path
+  const int g = p->hq / p->hkv;
+  if (D == 128 && !(p->flags & BF_FLAG_MMA_SYNC) && p->hq % 2 == 0 && g % 2 == 0) {
+    // tcgen05 ping-pong path: two heads of one GQA group per CTA
+    bf::Tc2Args ta;
+    std::memset(&ta, 0, sizeof(ta));
+    if (!make_k_map(&ta.qo_map, aa.Qo, L, batch * p->hq) || !make_k_map(&ta.ql_map, aa.Ql, L, batch * p->hq) ||
+        !make_k_map(&ta.ko_map, aa.Ko, L, batch * p->hkv) || !make_k_map(&ta.kl_map, aa.Kl, L, batch * p->hkv) ||
+        !make_v_map(&ta.v_map, aa.V, L, p->hkv, batch))
+      return BF_ERR_CUDA;
+    ta.out = aa.out;
+    ta.lse = aa.lse;
+    ta.L = L;
+    ta.hq = p->hq;
+    ta.hkv = p->hkv;
+    ta.batch = batch;
+    ta.w0 = aa.w0;
+    ta.scale_log2 = aa.scale_log2;
+    constexpr int smem = bf::attn_tc2_smem_bytes();
+    const long long n_cta = static_cast<long long>((L + bf::tc::BM - 1) / bf::tc::BM) * (p->hq / 2) * batch;
+    if (n_cta > 0x7fffffffLL) return BF_ERR_UNSUPPORTED;
+    auto kern = plan.bif ? bf::attn_tc2_kernel<true> : bf::attn_tc2_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) {
+      kern<<<static_cast<unsigned>(n_cta), bf::tc2::NTHREADS2, smem, st>>>(ta);
+      e = cudaGetLastError();
+    }
+  } else if (D == 128 && !(p->flags & BF_FLAG_MMA_SYNC)) {
+    // tcgen05 single-tile path (odd GQA groups)
     bf::TcArgs ta;
     std::memset(&ta, 0, sizeof(ta));
     if (!make_k_map(&ta.ko_map, aa.Ko, L, batch * p->hkv) || !make_k_map(&ta.kl_map, aa.Kl, L, batch * p->hkv) ||

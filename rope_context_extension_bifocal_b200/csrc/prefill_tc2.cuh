@@ -1,0 +1,471 @@
+// Bifocal causal prefill, tcgen05 ping-pong form: two query tiles per CTA (D = 128).
+//
+// One CTA owns the same 128 query rows of two heads of one GQA group, so both tiles use
+// every K and V tile it loads. Tensor memory (512 columns):
+//   [  0, 128) S_A / P_A   [128, 256) S_B / P_B   [256, 384) O_A   [384, 512) O_B
+// Q of both heads sits in shared memory (the A operand of QK^T), K/V tiles (128 keys)
+// arrive by TMA into a ring of four 32 KB slots.
+//
+// Warp roles: warps 0..3 = softmax of tile A, warps 4..7 = softmax of tile B (a thread owns
+// one query row; warp w reads TMEM lanes 32*(w%4)..), warp 8 = TMA producer, warp 9 = MMA
+// issuer (one thread). The MMA thread issues, per visit v,
+//   PV_A(v), QK_A(v+1), PV_B(v), QK_B(v+1)
+// so while one tile's softmax runs, the tensor core works on the other tile: the two
+// softmax groups never wait for each other.
+//
+// Visit order. Every key tile is scored with the branch that owns its pairs (ai-feeds
+// summary of Jet-Long, 方法 key modules 1 and 3): the long-range RoPE forms when all pairs
+// satisfy i - j >= w0, the original forms when all satisfy i - j < w0, and both (with
+// complementary masks) when the band edge crosses the tile. The online softmax does not
+// depend on the order of its terms, so the CTA takes all long-range visits first, then
+// reloads Q with its original-RoPE form once, then takes the local visits. That keeps
+// one Q form in shared memory at a time.
+#pragma once
+#include "common.cuh"
+#include "prefill_tc.cuh"
+
+namespace bf {
+namespace tc2 {
+
+using namespace tc;
+constexpr int NSLOT2 = 4;
+constexpr int NTHREADS2 = 320;  // 8 softmax warps, TMA warp, MMA warp
+constexpr uint32_t Q_BYTES = 32768;  // one Q tile, same layout as a K tile
+constexpr uint32_t COL_SA = 0, COL_SB = 128, COL_OA = 256, COL_OB = 384;
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "setp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+      "}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]));
+}
+
+__device__ __forceinline__ int floordiv(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
+
+// Visit schedule of one query tile: n_lf fully long tiles (0..n_lf-1), then n_b band-edge
+// tiles, then the rest fully local. Visits: long tiles, long half of band tiles, [Q reload],
+// local half of band tiles (when w0 > 0), local tiles.
+struct Schedule {
+  int n_kt, n_lf, n_b, n_bl, n_of;
+  __device__ __forceinline__ int n_long() const { return n_lf + n_b; }
+  __device__ __forceinline__ int total() const { return n_lf + n_b + n_bl + n_of; }
+  __device__ __forceinline__ void visit(int v, int& t, int& kind) const {
+    if (v < n_lf) {
+      t = v;
+      kind = LONG_FULL;
+    } else if (v < n_lf + n_b) {
+      t = v;  // band tiles follow the long tiles
+      kind = LONG_ONLY;
+    } else if (v < n_lf + n_b + n_bl) {
+      t = n_lf + (v - n_lf - n_b);
+      kind = ORIG_LOCAL;
+    } else {
+      t = n_lf + n_b + (v - n_lf - n_b - n_bl);
+      kind = ORIG_FULL;
+    }
+  }
+};
+
+template <bool BIFOCAL>
+__device__ __forceinline__ Schedule make_schedule(int i0, int n_kt, int w0) {
+  Schedule s;
+  s.n_kt = n_kt;
+  if (!BIFOCAL) {
+    s.n_lf = s.n_b = s.n_bl = 0;
+    s.n_of = n_kt;
+    return s;
+  }
+  const int A = floordiv(i0 - (BN - 1) - w0, BN);      // tiles t <= A: every pair long-range
+  const int C = floordiv(i0 + (BM - 1) - w0, BN) + 1;  // tiles t >= C: every pair local
+  s.n_lf = min(max(A + 1, 0), n_kt);
+  s.n_b = max(min(C, n_kt) - s.n_lf, 0);
+  s.n_bl = w0 > 0 ? s.n_b : 0;
+  s.n_of = n_kt - s.n_lf - s.n_b;
+  return s;
+}
+
+}  // namespace tc2
+
+struct Tc2Args {
+  CUtensorMap qo_map;  // fp16 [b*hq][L][128], box (64, 128, 1), 128B swizzle
+  CUtensorMap ql_map;
+  CUtensorMap ko_map;  // fp16 [b*hkv][L][128]
+  CUtensorMap kl_map;
+  CUtensorMap v_map;   // bf16 [b][L][hkv][128], box (64, 1, 128, 1)
+  __nv_bfloat16* out;  // [b, L, hq, 128]
+  float* lse;          // [b, hq, L] or null
+  int L, hq, hkv, batch, w0;
+  float scale_log2;
+};
+
+template <bool BIFOCAL>
+__global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __grid_constant__ Tc2Args a) {
+  using namespace tc2;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ uint64_t full[NSLOT2], empty[NSLOT2], s_full[2], p_ready[2], o_done[2], q_full, q_free, mma_drain;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_qt = (a.L + BM - 1) / BM;
+  const int pairs = a.hq / 2;
+  const int per_tile = pairs * a.batch;
+  const int qt = n_qt - 1 - static_cast<int>(blockIdx.x) / per_tile;  // heaviest first
+  const int rem = static_cast<int>(blockIdx.x) % per_tile;
+  const int hp = rem % pairs, b = rem / pairs;
+  const int h0 = 2 * hp;  // heads h0 (tile A) and h0 + 1 (tile B), same kv head
+  const int kvh = h0 / (a.hq / a.hkv);
+  const int i0 = qt * BM;
+  const int n_kt = (min(i0 + BM, a.L) + BN - 1) / BN;
+  const Schedule sch = make_schedule<BIFOCAL>(i0, n_kt, a.w0);
+  const int nv = sch.total();
+  const bool has_long = sch.n_long() > 0;
+  const bool has_orig = sch.n_bl + sch.n_of > 0;
+  const bool reload_q = has_long && has_orig;
+  const int v_sw = sch.n_long();  // first local visit (when reload_q)
+  const uint32_t qbase = smem_u32(smem);                  // Q_A, Q_B
+  const uint32_t slots = qbase + 2 * Q_BYTES;             // K/V ring
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int i = 0; i < NSLOT2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_ready[i], 4);
+      mbar_init(&o_done[i], 1);
+    }
+    mbar_init(&q_full, 1);
+    mbar_init(&q_free, 1);
+    mbar_init(&mma_drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_sh)),
+                 "r"(NCOLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&a.qo_map);
+      prefetch_tensormap(&a.ko_map);
+      prefetch_tensormap(&a.v_map);
+      if (BIFOCAL) {
+        prefetch_tensormap(&a.ql_map);
+        prefetch_tensormap(&a.kl_map);
+      }
+      const int qrow = b * a.hq + h0;
+      auto load_q = [&](const CUtensorMap* m) {
+        mbar_arrive_expect_tx(&q_full, 2 * Q_BYTES);
+        for (int x = 0; x < 2; ++x) {
+          uint8_t* dst = smem + x * Q_BYTES;
+          tma_load_3d(dst, m, &q_full, 0, i0, qrow + x);
+          tma_load_3d(dst + HALF_BYTES, m, &q_full, 64, i0, qrow + x);
+        }
+      };
+      load_q(has_long ? &a.ql_map : &a.qo_map);
+      const int krow = b * a.hkv + kvh;
+      int n = 0;
+      bool ok = true;
+      for (int v = 0; v < nv && ok; ++v) {
+        if (reload_q && v == v_sw) {
+          // every QK^T with the long-range Q has finished reading it
+          if (!mbar_wait_abortable(&q_free, 0, 12, &s_abort)) {
+            ok = false;
+            break;
+          }
+          load_q(&a.qo_map);
+        }
+        int t, kind;
+        sch.visit(v, t, kind);
+        const bool lng = kind == LONG_FULL || kind == LONG_ONLY;
+        for (int x = 0; x < 2; ++x, ++n) {
+          const int slot = n % NSLOT2, use = n / NSLOT2;
+          if (use > 0 && !mbar_wait_abortable(&empty[slot], (use - 1) & 1, 10, &s_abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[slot], SLOT_BYTES);
+          uint8_t* dst = smem + 2 * Q_BYTES + slot * SLOT_BYTES;
+          if (x == 0) {
+            const CUtensorMap* m = lng ? &a.kl_map : &a.ko_map;
+            tma_load_3d(dst, m, &full[slot], 0, t * BN, krow);
+            tma_load_3d(dst + HALF_BYTES, m, &full[slot], 64, t * BN, krow);
+          } else {
+            tma_load_4d(dst, &a.v_map, &full[slot], 0, kvh, t * BN, b);
+            tma_load_4d(dst + HALF_BYTES, &a.v_map, &full[slot], 64, kvh, t * BN, b);
+          }
+        }
+      }
+      // drain: every fill issued must have landed before the CTA may exit
+      const int first = n > NSLOT2 ? n - NSLOT2 : 0;
+      for (int k = first; k < n; ++k) mbar_wait(&full[k % NSLOT2], (k / NSLOT2) & 1, 11);
+      mbar_wait(&q_full, reload_q ? 1 : 0, 13);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nv > 0) {
+      bool ok = mbar_wait_abortable(&q_full, 0, 20, &s_abort);
+      fence_after();
+      auto kslot = [&](int v) { return (2 * v) % NSLOT2; };
+      auto vslot = [&](int v) { return (2 * v + 1) % NSLOT2; };
+      auto kphase = [&](int v) { return static_cast<uint32_t>(((2 * v) / NSLOT2) & 1); };
+      auto vphase = [&](int v) { return static_cast<uint32_t>(((2 * v + 1) / NSLOT2) & 1); };
+      auto qk = [&](int x, int v) {
+        const uint32_t ks = slots + kslot(v) * SLOT_BYTES;
+        const uint32_t qs = qbase + x * Q_BYTES;
+        const uint32_t d = tmem + (x == 0 ? COL_SA : COL_SB);
+#pragma unroll 1
+        for (int kk = 0; kk < 8; ++kk) mma_ss(d, k_desc(qs, kk), k_desc(ks, kk), IDESC_QK, kk > 0);
+        mma_commit(&s_full[x]);
+      };
+      auto pv = [&](int x, int v) {
+        const uint32_t vs = slots + vslot(v) * SLOT_BYTES;
+        const uint32_t p_col = tmem + (x == 0 ? COL_SA : COL_SB);
+        const uint32_t o_col = tmem + (x == 0 ? COL_OA : COL_OB);
+#pragma unroll 1
+        for (int kk = 0; kk < 8; ++kk) mma_ts(o_col, p_col + kk * 8, v_desc(vs, kk), IDESC_PV, (v > 0) || kk > 0);
+        mma_commit(&o_done[x]);
+      };
+      // visit 0: S_A, S_B
+      if (ok) ok = mbar_wait_abortable(&full[kslot(0)], kphase(0), 21, &s_abort);
+      if (ok) {
+        fence_after();
+        qk(0, 0);
+        qk(1, 0);
+        mma_commit(&empty[kslot(0)]);
+        if (reload_q && v_sw == 1) mma_commit(&q_free);
+      }
+      for (int v = 0; v < nv && ok; ++v) {
+        // O_A += P_A(v) V(v)
+        if (!mbar_wait_abortable(&p_ready[0], v & 1, 22, &s_abort) ||
+            !mbar_wait_abortable(&full[vslot(v)], vphase(v), 23, &s_abort)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        pv(0, v);
+        const bool more = v + 1 < nv;
+        if (more) {
+          if (reload_q && v + 1 == v_sw && !mbar_wait_abortable(&q_full, 1, 24, &s_abort)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait_abortable(&full[kslot(v + 1)], kphase(v + 1), 25, &s_abort)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          qk(0, v + 1);  // S_A is free: PV_A(v) was issued before
+        }
+        // O_B += P_B(v) V(v)
+        if (!mbar_wait_abortable(&p_ready[1], v & 1, 26, &s_abort)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        pv(1, v);
+        mma_commit(&empty[vslot(v)]);
+        if (more) {
+          qk(1, v + 1);
+          mma_commit(&empty[kslot(v + 1)]);
+          if (reload_q && v + 2 == v_sw) mma_commit(&q_free);
+        }
+      }
+      // every MMA issued has finished before teardown
+      mma_commit(&mma_drain);
+      mbar_wait(&mma_drain, 0, 27);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax warps: 0..3 tile A, 4..7 tile B
+    const int x = warp >> 2;        // tile
+    const int quad = warp & 3;      // TMEM lane quadrant this warp may access
+    const int r = quad * 32 + lane;
+    const int i = i0 + r;
+    const int h = h0 + x;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t s_col = lane_addr + (x == 0 ? COL_SA : COL_SB);
+    const uint32_t o_col = lane_addr + (x == 0 ? COL_OA : COL_OB);
+    const float sc = a.scale_log2;
+    float m_ref = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    for (int v = 0; v < nv && ok; ++v) {
+      int t, kind;
+      sch.visit(v, t, kind);
+      const int j0 = t * BN;
+      // every lane waits; the result is made warp-uniform because the TMEM accesses below
+      // are warp-collective (.sync.aligned)
+      if (!__all_sync(0xffffffffu, mbar_wait_abortable(&s_full[x], v & 1, 30, &s_abort))) {
+        ok = false;
+        break;
+      }
+      fence_after();
+      const bool masked = kind != LONG_FULL && (kind != ORIG_FULL || j0 + BN - 1 > i0);
+      const int lo = (kind == LONG_ONLY) ? a.w0 : 0;            // keep lo <= i - j
+      const int hi = (kind == ORIG_LOCAL) ? a.w0 : 0x7fffffff;  //      and i - j < hi
+      float alpha = 1.f, rs = 0.f;
+      bool grow = false;
+      uint32_t pk[64];  // P of the whole row, bf16 pairs; stored to TMEM once it is final
+      // Fast path (unmasked visits once the row has a reference): one pass with the current
+      // reference m_ref. m_ref never exceeds the running max, so every P term is bounded by
+      // 2^(running max - m_ref); the row sum bounds them all, and a sum above 2^24 (or not
+      // finite) sends the visit to the exact two-pass path below.
+      bool exact = masked || m_ref == -INFINITY;
+      if (!exact) {
+        const float neg_ref = -m_ref;
+        float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          float s[32];
+          tmem_ld32(s_col + c0, s);
+          wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = fast_exp2(fmaf(s[c], sc, neg_ref)), p1 = fast_exp2(fmaf(s[c + 1], sc, neg_ref));
+            r8[(c >> 1) & 7] += p0 + p1;
+            pk[(c0 + c) >> 1] = pack_bf16x2(p0, p1);
+          }
+        }
+        rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+        exact = !(rs <= 16777216.f);
+      }
+      if (exact) {
+        // pass 1: raw row max over the 128 columns
+        float m8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m8[u] = -INFINITY;
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          float s[32];
+          tmem_ld32(s_col + c0, s);
+          wait_ld();
+          if (masked) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const int d = i - (j0 + c0 + c);
+              s[c] = (d >= lo && d < hi) ? s[c] : -INFINITY;
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 32; c += 8)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) m8[u] = fmaxf(m8[u], s[c + u]);
+        }
+        const float mx =
+            fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
+            sc;
+        // lazy rescale: a row keeps its reference unless its max grew by more than the threshold
+        if (mx > m_ref + RESCALE_THRESHOLD || (m_ref == -INFINITY && mx > -INFINITY)) {
+          alpha = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mx);
+          grow = m_ref != -INFINITY;  // O already holds this row's earlier terms
+          m_ref = mx;
+        }
+        const float neg_ref = (m_ref == -INFINITY) ? 0.f : -m_ref;
+        // pass 2: P = exp2(s * scale - ref)
+        float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          float s[32];
+          tmem_ld32(s_col + c0, s);
+          wait_ld();
+          if (masked) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const int d = i - (j0 + c0 + c);
+              s[c] = (d >= lo && d < hi) ? s[c] : -INFINITY;
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = fast_exp2(fmaf(s[c], sc, neg_ref)), p1 = fast_exp2(fmaf(s[c + 1], sc, neg_ref));
+            r8[(c >> 1) & 7] += p0 + p1;
+            pk[(c0 + c) >> 1] = pack_bf16x2(p0, p1);
+          }
+        }
+        rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+      }
+      l_sum = l_sum * alpha + rs;
+      tmem_st32(s_col, pk);       // P over the first 64 columns of the S buffer
+      tmem_st32(s_col + 32, pk + 32);
+      // O_x must hold PV(v-1) before it is rescaled and before PV(v) adds to it
+      if (v >= 1) {
+        if (!__all_sync(0xffffffffu, mbar_wait_abortable(&o_done[x], (v - 1) & 1, 31, &s_abort))) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        if (__any_sync(0xffffffffu, grow)) {  // warp-uniform; rows that need none scale by 1
+          const float f = grow ? alpha : 1.f;
+#pragma unroll 1
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            float ov[32];
+            tmem_ld32(o_col + c0, ov);
+            wait_ld();
+            uint32_t ou[32];
+#pragma unroll
+            for (int u = 0; u < 32; ++u) ou[u] = __float_as_uint(ov[u] * f);
+            tmem_st32(o_col + c0, ou);
+          }
+        }
+      }
+      wait_st();
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready[x]);
+    }
+    // epilogue: O / l -> bf16, LSE
+    if (ok && nv > 0 && __all_sync(0xffffffffu, mbar_wait_abortable(&o_done[x], (nv - 1) & 1, 32, &s_abort))) {
+      fence_after();
+      const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      __nv_bfloat16* orow = a.out + ((static_cast<long long>(b) * a.L + i) * a.hq + h) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        float ov[32];
+        tmem_ld32(o_col + c0, ov);
+        wait_ld();
+        if (i < a.L) {
+#pragma unroll
+          for (int u = 0; u < 32; u += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(ov[u] * inv, ov[u + 1] * inv);
+            w.y = pack_bf16x2(ov[u + 2] * inv, ov[u + 3] * inv);
+            w.z = pack_bf16x2(ov[u + 4] * inv, ov[u + 5] * inv);
+            w.w = pack_bf16x2(ov[u + 6] * inv, ov[u + 7] * inv);
+            *reinterpret_cast<uint4*>(orow + c0 + u) = w;
+          }
+        }
+      }
+      if (a.lse && i < a.L)
+        a.lse[(static_cast<long long>(b) * a.hq + h) * a.L + i] = (m_ref + __log2f(l_sum)) * 0.69314718055994530942f;
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 9) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NCOLS));
+}
+
+constexpr int attn_tc2_smem_bytes() { return 2 * tc2::Q_BYTES + tc2::NSLOT2 * tc::SLOT_BYTES; }
+
+}  // namespace bf
