@@ -101,6 +101,23 @@ bool make_cache_map(CUtensorMap* map, const void* base, int cap, int hkv, int D,
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Launch with programmatic stream serialisation: the kernel may start while the previous
+// kernel on the stream is still running; it synchronises with griddepcontrol.wait.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Rotated key forms [rows = b*hkv][L][128] fp16, box (64, 128, 1), 128B swizzle.
 bool make_k_map(CUtensorMap* map, const void* base, int L, int rows) {
   auto fn = encode_fn();
@@ -415,25 +432,33 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
   std::memcpy(da.omega_corr, rope.omega_corr, sizeof(da.omega_corr));
   const dim3 grid(n_split, head_groups);
   cudaError_t e;
+  // the partial and combine kernels overlap their launch with the kernel before them
   if (D == 128) {
     constexpr int smem = bf::decode_smem_bytes<128>();
     e = cudaFuncSetAttribute(bf::decode_partial_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) bf::decode_partial_kernel<128><<<grid, bf::decode_threads<128>(), smem, st>>>(da);
+    if (e == cudaSuccess)
+      e = launch_pdl(bf::decode_partial_kernel<128>, grid, dim3(bf::decode_threads<128>()), smem, st, da);
   } else {
     constexpr int smem = bf::decode_smem_bytes<64>();
     e = cudaFuncSetAttribute(bf::decode_partial_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) bf::decode_partial_kernel<64><<<grid, bf::decode_threads<64>(), smem, st>>>(da);
+    if (e == cudaSuccess)
+      e = launch_pdl(bf::decode_partial_kernel<64>, grid, dim3(bf::decode_threads<64>()), smem, st, da);
   }
-  if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
+  if (e != cudaSuccess) return BF_ERR_CUDA;
 
   // 3. combine
+  const float* po = da.part_o;
+  const float* pml = da.part_ml;
+  const int nparts = 2 * n_split;
+  const int hq = p->hq;
+  bf16* o16 = static_cast<bf16*>(out);
   if (D == 128)
-    bf::decode_combine_kernel<128><<<p->hq, 128, 0, st>>>(da.part_o, da.part_ml, 2 * n_split, p->hq,
-                                                         static_cast<bf16*>(out), lse);
+    e = launch_pdl(bf::decode_combine_kernel<128>, dim3(p->hq), dim3(128 * bf::COMBINE_GROUPS), 0, st, po, pml, nparts,
+                   hq, o16, lse);
   else
-    bf::decode_combine_kernel<64><<<p->hq, 64, 0, st>>>(da.part_o, da.part_ml, 2 * n_split, p->hq,
-                                                       static_cast<bf16*>(out), lse);
-  return cudaGetLastError() == cudaSuccess ? BF_OK : BF_ERR_CUDA;
+    e = launch_pdl(bf::decode_combine_kernel<64>, dim3(p->hq), dim3(64 * bf::COMBINE_GROUPS), 0, st, po, pml, nparts,
+                   hq, o16, lse);
+  return e == cudaSuccess ? BF_OK : BF_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------ allocation-free decode

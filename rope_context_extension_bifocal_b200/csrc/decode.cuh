@@ -71,6 +71,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   uint64_t* empty = full + NST;
   __shared__ int s_abort;  // set when a bounded wait expires: later waits return at once
 
+  pdl_launch_dependents();  // the combine may start its prologue; it waits for this grid's writes
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head0 = blockIdx.y * HPC;
   const int nheads = min(HPC, a.hkv - head0);
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
     if (lane == 0) {
       prefetch_tensormap(&a.kmap);
       prefetch_tensormap(&a.vmap);
+      pdl_wait();  // the append kernel has written the new cache row
       const uint32_t bytes = 2u * nheads * HALVES * HEAD_TILE;
       for (int s = 0; s < nstage; ++s) {
         const int st = s % NST;
@@ -346,23 +348,56 @@ constexpr int decode_threads() {
   return (2 * dec::HPC + 3) * 32;  // consumers, TMA warp, two table warps
 }
 
-// Log-sum-exp merge of the split partials: one CTA per query head, one thread per d.
+// Log-sum-exp merge of the split partials: one CTA per query head. The global max comes
+// from a warp-cooperative reduction over the partial maxima; then COMBINE_GROUPS groups of
+// D threads each sum a strided share of the partials for their d, and shared memory adds
+// the groups.
+constexpr int COMBINE_GROUPS = 4;
+
 template <int D>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ part_o,
-                                                            const float* __restrict__ part_ml, int n_split, int hq,
-                                                            __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
-  const int h = blockIdx.x, d = threadIdx.x;
+__global__ void __launch_bounds__(D * COMBINE_GROUPS) decode_combine_kernel(
+    const float* __restrict__ part_o, const float* __restrict__ part_ml, int n_split, int hq,
+    __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  __shared__ float red_acc[COMBINE_GROUPS][D];
+  __shared__ float red_l[COMBINE_GROUPS];
+  __shared__ float warp_max[D * COMBINE_GROUPS / 32];
+  pdl_wait();  // the partials of the previous kernel are complete and visible
+  const int h = blockIdx.x, tid = threadIdx.x;
+  const int d = tid % D, grp = tid / D;
+  const int lane = tid & 31, warp = tid >> 5;
+  // global max of the partial maxima
   float M = -INFINITY;
-  for (int s = 0; s < n_split; ++s) M = fmaxf(M, part_ml[(s * hq + h) * 2]);
+  for (int s = tid; s < n_split; s += D * COMBINE_GROUPS) M = fmaxf(M, part_ml[(static_cast<long long>(s) * hq + h) * 2]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) warp_max[warp] = M;
+  __syncthreads();
+  M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < D * COMBINE_GROUPS / 32; ++w) M = fmaxf(M, warp_max[w]);
   const float ref = (M == -INFINITY) ? 0.f : M;
-  float lsum = 0.f, acc = 0.f;
-  for (int s = 0; s < n_split; ++s) {
-    const float w = exp2f(part_ml[(s * hq + h) * 2] - ref);
-    lsum += w * part_ml[(s * hq + h) * 2 + 1];
-    acc += w * part_o[(static_cast<long long>(s) * hq + h) * D + d];
+  // this group's share of the partials
+  float acc = 0.f, lsum = 0.f;
+#pragma unroll 4
+  for (int s = grp; s < n_split; s += COMBINE_GROUPS) {
+    const long long row = static_cast<long long>(s) * hq + h;
+    const float w = exp2f(part_ml[row * 2] - ref);
+    lsum += w * part_ml[row * 2 + 1];
+    acc += w * part_o[row * D + d];
   }
-  out[h * D + d] = __float2bfloat16(acc / lsum);
-  if (lse && d == 0) lse[h] = (M + log2f(lsum)) * 0.69314718055994530942f;
+  red_acc[grp][d] = acc;
+  if (d == 0) red_l[grp] = lsum;
+  __syncthreads();
+  if (grp == 0) {
+    float a = 0.f, l = 0.f;
+#pragma unroll
+    for (int g = 0; g < COMBINE_GROUPS; ++g) {
+      a += red_acc[g][d];
+      l += red_l[g];
+    }
+    out[h * D + d] = __float2bfloat16(a / l);
+    if (lse && d == 0) lse[h] = (M + log2f(l)) * 0.69314718055994530942f;
+  }
 }
 
 // Append: cache row p <- (R_orig(p) k_new, v_new). One warp per kv head.
@@ -378,6 +413,7 @@ struct AppendArgs {
 template <int D>
 __global__ void decode_append_kernel(const __grid_constant__ AppendArgs a) {
   constexpr int P = D / 2;
+  pdl_launch_dependents();  // the partial kernel may start its prologue; its TMA thread waits for us
   const int h = blockIdx.x, lane = threadIdx.x;
   const __nv_bfloat16* kr = a.k_new + h * D;
   __nv_bfloat16* kd = a.kcache + (static_cast<long long>(a.p) * a.hkv + h) * D;
