@@ -98,12 +98,14 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
     if (lane == 0) {
       prefetch_tensormap(&a.kmap);
       prefetch_tensormap(&a.vmap);
-      pdl_wait();  // the append kernel has written the new cache row
       const uint32_t bytes = 2u * nheads * HALVES * HEAD_TILE;
       for (int s = 0; s < nstage; ++s) {
         const int st = s % NST;
         if (s >= NST && !mbar_wait_abortable(&empty[st], ((s / NST) - 1) & 1, 1, &s_abort)) break;
         const int j0 = jbeg + s * KB;
+        // Only row p (the new token) comes from the append kernel; every other row was in the
+        // cache before this step, so only the stage holding p waits for that grid.
+        if (j0 + KB > p) pdl_wait();
         mbar_arrive_expect_tx(&full[st], bytes);
         for (int hh = 0; hh < nheads; ++hh)
           for (int hf = 0; hf < HALVES; ++hf) {
@@ -413,7 +415,7 @@ struct AppendArgs {
 template <int D>
 __global__ void decode_append_kernel(const __grid_constant__ AppendArgs a) {
   constexpr int P = D / 2;
-  pdl_launch_dependents();  // the partial kernel may start its prologue; its TMA thread waits for us
+  pdl_launch_dependents();  // the partial kernel may start; only its stage holding row p waits for us
   const int h = blockIdx.x, lane = threadIdx.x;
   const __nv_bfloat16* kr = a.k_new + h * D;
   __nv_bfloat16* kd = a.kcache + (static_cast<long long>(a.p) * a.hkv + h) * D;

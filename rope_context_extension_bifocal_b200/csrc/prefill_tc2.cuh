@@ -8,7 +8,11 @@
 //
 // Warp roles: warps 0..3 = softmax of tile A, warps 4..7 = softmax of tile B (a thread owns
 // one query row; warp w reads TMEM lanes 32*(w%4)..), warp 8 = TMA producer, warp 9 = MMA
-// issuer (one thread). The MMA thread issues, per visit v,
+// issuer (one thread), warps 10..11 idle. Warps 8..11 form the third warpgroup only so that
+// it can hand registers to the softmax warpgroups (setmaxnreg works per warpgroup): with 384
+// threads the launch gives 168 registers per thread, the softmax rows need more than that to
+// hold a 32-column S chunk and the whole row's P without spilling. The MMA thread issues,
+// per visit v,
 //   PV_A(v), QK_A(v+1), PV_B(v), QK_B(v+1)
 // so while one tile's softmax runs, the tensor core works on the other tile: the two
 // softmax groups never wait for each other.
@@ -29,7 +33,7 @@ namespace tc2 {
 
 using namespace tc;
 constexpr int NSLOT2 = 4;
-constexpr int NTHREADS2 = 320;  // 8 softmax warps, TMA warp, MMA warp
+constexpr int NTHREADS2 = 384;  // 8 softmax warps, TMA warp, MMA warp, 2 idle warps (register donors)
 constexpr uint32_t Q_BYTES = 32768;  // one Q tile, same layout as a K tile
 constexpr uint32_t COL_SA = 0, COL_SB = 128, COL_OA = 256, COL_OB = 384;
 
@@ -164,139 +168,148 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
   fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tensormap(&a.qo_map);
-      prefetch_tensormap(&a.ko_map);
-      prefetch_tensormap(&a.v_map);
-      if (BIFOCAL) {
-        prefetch_tensormap(&a.ql_map);
-        prefetch_tensormap(&a.kl_map);
+  // Registers: launched at 168 per thread (384 threads). Warpgroup 2 (TMA, MMA, two idle
+  // warps) gives 96 of them back and the two softmax warpgroups take 48 more each:
+  // 2 * 128 * 216 + 128 * 72 = 384 * 168, so the increase never waits for registers that
+  // the block does not hold. Each role branch starts with its own setmaxnreg so that the
+  // compiler allocates each branch within its own limit.
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+    if (warp == 8) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        prefetch_tensormap(&a.qo_map);
+        prefetch_tensormap(&a.ko_map);
+        prefetch_tensormap(&a.v_map);
+        if (BIFOCAL) {
+          prefetch_tensormap(&a.ql_map);
+          prefetch_tensormap(&a.kl_map);
+        }
+        const int qrow = b * a.hq + h0;
+        auto load_q = [&](const CUtensorMap* m) {
+          mbar_arrive_expect_tx(&q_full, 2 * Q_BYTES);
+          for (int x = 0; x < 2; ++x) {
+            uint8_t* dst = smem + x * Q_BYTES;
+            tma_load_3d(dst, m, &q_full, 0, i0, qrow + x);
+            tma_load_3d(dst + HALF_BYTES, m, &q_full, 64, i0, qrow + x);
+          }
+        };
+        load_q(has_long ? &a.ql_map : &a.qo_map);
+        const int krow = b * a.hkv + kvh;
+        int n = 0;
+        bool ok = true;
+        for (int v = 0; v < nv && ok; ++v) {
+          if (reload_q && v == v_sw) {
+            // every QK^T with the long-range Q has finished reading it
+            if (!mbar_wait_abortable(&q_free, 0, 12, &s_abort)) {
+              ok = false;
+              break;
+            }
+            load_q(&a.qo_map);
+          }
+          int t, kind;
+          sch.visit(v, t, kind);
+          const bool lng = kind == LONG_FULL || kind == LONG_ONLY;
+          for (int x = 0; x < 2; ++x, ++n) {
+            const int slot = n % NSLOT2, use = n / NSLOT2;
+            if (use > 0 && !mbar_wait_abortable(&empty[slot], (use - 1) & 1, 10, &s_abort)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[slot], SLOT_BYTES);
+            uint8_t* dst = smem + 2 * Q_BYTES + slot * SLOT_BYTES;
+            if (x == 0) {
+              const CUtensorMap* m = lng ? &a.kl_map : &a.ko_map;
+              tma_load_3d(dst, m, &full[slot], 0, t * BN, krow);
+              tma_load_3d(dst + HALF_BYTES, m, &full[slot], 64, t * BN, krow);
+            } else {
+              tma_load_4d(dst, &a.v_map, &full[slot], 0, kvh, t * BN, b);
+              tma_load_4d(dst + HALF_BYTES, &a.v_map, &full[slot], 64, kvh, t * BN, b);
+            }
+          }
+        }
+        // drain: every fill issued must have landed before the CTA may exit
+        const int first = n > NSLOT2 ? n - NSLOT2 : 0;
+        for (int k = first; k < n; ++k) mbar_wait(&full[k % NSLOT2], (k / NSLOT2) & 1, 11);
+        mbar_wait(&q_full, reload_q ? 1 : 0, 13);
       }
-      const int qrow = b * a.hq + h0;
-      auto load_q = [&](const CUtensorMap* m) {
-        mbar_arrive_expect_tx(&q_full, 2 * Q_BYTES);
-        for (int x = 0; x < 2; ++x) {
-          uint8_t* dst = smem + x * Q_BYTES;
-          tma_load_3d(dst, m, &q_full, 0, i0, qrow + x);
-          tma_load_3d(dst + HALF_BYTES, m, &q_full, 64, i0, qrow + x);
-        }
-      };
-      load_q(has_long ? &a.ql_map : &a.qo_map);
-      const int krow = b * a.hkv + kvh;
-      int n = 0;
-      bool ok = true;
-      for (int v = 0; v < nv && ok; ++v) {
-        if (reload_q && v == v_sw) {
-          // every QK^T with the long-range Q has finished reading it
-          if (!mbar_wait_abortable(&q_free, 0, 12, &s_abort)) {
-            ok = false;
-            break;
-          }
-          load_q(&a.qo_map);
-        }
-        int t, kind;
-        sch.visit(v, t, kind);
-        const bool lng = kind == LONG_FULL || kind == LONG_ONLY;
-        for (int x = 0; x < 2; ++x, ++n) {
-          const int slot = n % NSLOT2, use = n / NSLOT2;
-          if (use > 0 && !mbar_wait_abortable(&empty[slot], (use - 1) & 1, 10, &s_abort)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[slot], SLOT_BYTES);
-          uint8_t* dst = smem + 2 * Q_BYTES + slot * SLOT_BYTES;
-          if (x == 0) {
-            const CUtensorMap* m = lng ? &a.kl_map : &a.ko_map;
-            tma_load_3d(dst, m, &full[slot], 0, t * BN, krow);
-            tma_load_3d(dst + HALF_BYTES, m, &full[slot], 64, t * BN, krow);
-          } else {
-            tma_load_4d(dst, &a.v_map, &full[slot], 0, kvh, t * BN, b);
-            tma_load_4d(dst + HALF_BYTES, &a.v_map, &full[slot], 64, kvh, t * BN, b);
-          }
-        }
-      }
-      // drain: every fill issued must have landed before the CTA may exit
-      const int first = n > NSLOT2 ? n - NSLOT2 : 0;
-      for (int k = first; k < n; ++k) mbar_wait(&full[k % NSLOT2], (k / NSLOT2) & 1, 11);
-      mbar_wait(&q_full, reload_q ? 1 : 0, 13);
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nv > 0) {
-      bool ok = mbar_wait_abortable(&q_full, 0, 20, &s_abort);
-      fence_after();
-      auto kslot = [&](int v) { return (2 * v) % NSLOT2; };
-      auto vslot = [&](int v) { return (2 * v + 1) % NSLOT2; };
-      auto kphase = [&](int v) { return static_cast<uint32_t>(((2 * v) / NSLOT2) & 1); };
-      auto vphase = [&](int v) { return static_cast<uint32_t>(((2 * v + 1) / NSLOT2) & 1); };
-      auto qk = [&](int x, int v) {
-        const uint32_t ks = slots + kslot(v) * SLOT_BYTES;
-        const uint32_t qs = qbase + x * Q_BYTES;
-        const uint32_t d = tmem + (x == 0 ? COL_SA : COL_SB);
-#pragma unroll 1
-        for (int kk = 0; kk < 8; ++kk) mma_ss(d, k_desc(qs, kk), k_desc(ks, kk), IDESC_QK, kk > 0);
-        mma_commit(&s_full[x]);
-      };
-      auto pv = [&](int x, int v) {
-        const uint32_t vs = slots + vslot(v) * SLOT_BYTES;
-        const uint32_t p_col = tmem + (x == 0 ? COL_SA : COL_SB);
-        const uint32_t o_col = tmem + (x == 0 ? COL_OA : COL_OB);
-#pragma unroll 1
-        for (int kk = 0; kk < 8; ++kk) mma_ts(o_col, p_col + kk * 8, v_desc(vs, kk), IDESC_PV, (v > 0) || kk > 0);
-        mma_commit(&o_done[x]);
-      };
-      // visit 0: S_A, S_B
-      if (ok) ok = mbar_wait_abortable(&full[kslot(0)], kphase(0), 21, &s_abort);
-      if (ok) {
+    } else if (warp == 9) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0 && nv > 0) {
+        bool ok = mbar_wait_abortable(&q_full, 0, 20, &s_abort);
         fence_after();
-        qk(0, 0);
-        qk(1, 0);
-        mma_commit(&empty[kslot(0)]);
-        if (reload_q && v_sw == 1) mma_commit(&q_free);
-      }
-      for (int v = 0; v < nv && ok; ++v) {
-        // O_A += P_A(v) V(v)
-        if (!mbar_wait_abortable(&p_ready[0], v & 1, 22, &s_abort) ||
-            !mbar_wait_abortable(&full[vslot(v)], vphase(v), 23, &s_abort)) {
-          ok = false;
-          break;
+        auto kslot = [&](int v) { return (2 * v) % NSLOT2; };
+        auto vslot = [&](int v) { return (2 * v + 1) % NSLOT2; };
+        auto kphase = [&](int v) { return static_cast<uint32_t>(((2 * v) / NSLOT2) & 1); };
+        auto vphase = [&](int v) { return static_cast<uint32_t>(((2 * v + 1) / NSLOT2) & 1); };
+        auto qk = [&](int x, int v) {
+          const uint32_t ks = slots + kslot(v) * SLOT_BYTES;
+          const uint32_t qs = qbase + x * Q_BYTES;
+          const uint32_t d = tmem + (x == 0 ? COL_SA : COL_SB);
+#pragma unroll 1
+          for (int kk = 0; kk < 8; ++kk) mma_ss(d, k_desc(qs, kk), k_desc(ks, kk), IDESC_QK, kk > 0);
+          mma_commit(&s_full[x]);
+        };
+        auto pv = [&](int x, int v) {
+          const uint32_t vs = slots + vslot(v) * SLOT_BYTES;
+          const uint32_t p_col = tmem + (x == 0 ? COL_SA : COL_SB);
+          const uint32_t o_col = tmem + (x == 0 ? COL_OA : COL_OB);
+#pragma unroll 1
+          for (int kk = 0; kk < 8; ++kk) mma_ts(o_col, p_col + kk * 8, v_desc(vs, kk), IDESC_PV, (v > 0) || kk > 0);
+          mma_commit(&o_done[x]);
+        };
+        // visit 0: S_A, S_B
+        if (ok) ok = mbar_wait_abortable(&full[kslot(0)], kphase(0), 21, &s_abort);
+        if (ok) {
+          fence_after();
+          qk(0, 0);
+          qk(1, 0);
+          mma_commit(&empty[kslot(0)]);
+          if (reload_q && v_sw == 1) mma_commit(&q_free);
         }
-        fence_after();
-        pv(0, v);
-        const bool more = v + 1 < nv;
-        if (more) {
-          if (reload_q && v + 1 == v_sw && !mbar_wait_abortable(&q_full, 1, 24, &s_abort)) {
-            ok = false;
-            break;
-          }
-          if (!mbar_wait_abortable(&full[kslot(v + 1)], kphase(v + 1), 25, &s_abort)) {
+        for (int v = 0; v < nv && ok; ++v) {
+          // O_A += P_A(v) V(v)
+          if (!mbar_wait_abortable(&p_ready[0], v & 1, 22, &s_abort) ||
+              !mbar_wait_abortable(&full[vslot(v)], vphase(v), 23, &s_abort)) {
             ok = false;
             break;
           }
           fence_after();
-          qk(0, v + 1);  // S_A is free: PV_A(v) was issued before
+          pv(0, v);
+          const bool more = v + 1 < nv;
+          if (more) {
+            if (reload_q && v + 1 == v_sw && !mbar_wait_abortable(&q_full, 1, 24, &s_abort)) {
+              ok = false;
+              break;
+            }
+            if (!mbar_wait_abortable(&full[kslot(v + 1)], kphase(v + 1), 25, &s_abort)) {
+              ok = false;
+              break;
+            }
+            fence_after();
+            qk(0, v + 1);  // S_A is free: PV_A(v) was issued before
+          }
+          // O_B += P_B(v) V(v)
+          if (!mbar_wait_abortable(&p_ready[1], v & 1, 26, &s_abort)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          pv(1, v);
+          mma_commit(&empty[vslot(v)]);
+          if (more) {
+            qk(1, v + 1);
+            mma_commit(&empty[kslot(v + 1)]);
+            if (reload_q && v + 2 == v_sw) mma_commit(&q_free);
+          }
         }
-        // O_B += P_B(v) V(v)
-        if (!mbar_wait_abortable(&p_ready[1], v & 1, 26, &s_abort)) {
-          ok = false;
-          break;
-        }
-        fence_after();
-        pv(1, v);
-        mma_commit(&empty[vslot(v)]);
-        if (more) {
-          qk(1, v + 1);
-          mma_commit(&empty[kslot(v + 1)]);
-          if (reload_q && v + 2 == v_sw) mma_commit(&q_free);
-        }
+        // every MMA issued has finished before teardown
+        mma_commit(&mma_drain);
+        mbar_wait(&mma_drain, 0, 27);
       }
-      // every MMA issued has finished before teardown
-      mma_commit(&mma_drain);
-      mbar_wait(&mma_drain, 0, 27);
     }
-  } else if (warp < 8) {
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
     // ------------------------------------------------------------ softmax warps: 0..3 tile A, 4..7 tile B
     const int x = warp >> 2;        // tile
     const int quad = warp & 3;      // TMEM lane quadrant this warp may access
@@ -332,8 +345,11 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
       // finite) sends the visit to the exact two-pass path below.
       bool exact = masked || m_ref == -INFINITY;
       if (!exact) {
-        const float neg_ref = -m_ref;
-        float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // pairs of columns go through the packed f32x2 FMA and add
+        const uint64_t sc2 = f2_pack(sc, sc), nref2 = f2_pack(-m_ref, -m_ref);
+        uint64_t r4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) r4[u] = f2_pack(0.f, 0.f);
 #pragma unroll
         for (int c0 = 0; c0 < 128; c0 += 32) {
           float s[32];
@@ -341,11 +357,16 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
           wait_ld();
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            const float p0 = fast_exp2(fmaf(s[c], sc, neg_ref)), p1 = fast_exp2(fmaf(s[c + 1], sc, neg_ref));
-            r8[(c >> 1) & 7] += p0 + p1;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sc2, nref2), x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            r4[(c >> 1) & 3] = f2_add(r4[(c >> 1) & 3], f2_pack(p0, p1));
             pk[(c0 + c) >> 1] = pack_bf16x2(p0, p1);
           }
         }
+        float r8[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) f2_unpack(r4[u], r8[2 * u], r8[2 * u + 1]);
         rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
         exact = !(rs <= 16777216.f);
       }
