@@ -169,12 +169,12 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
   const uint32_t tmem = tmem_base_sh;
 
   // Registers: launched at 168 per thread (384 threads). Warpgroup 2 (TMA, MMA, two idle
-  // warps) gives 96 of them back and the two softmax warpgroups take 48 more each:
-  // 2 * 128 * 216 + 128 * 72 = 384 * 168, so the increase never waits for registers that
-  // the block does not hold. Each role branch starts with its own setmaxnreg so that the
+  // warps) gives 72 of them back and the two softmax warpgroups take 32 more each:
+  // 2 * 128 * 200 + 128 * 96 = 63488 <= 384 * 168, so the increase never waits for registers
+  // that the block does not hold. Each role branch starts with its own setmaxnreg so that the
   // compiler allocates each branch within its own limit.
   if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 96;");
     if (warp == 8) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
@@ -242,20 +242,32 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
         auto vslot = [&](int v) { return (2 * v + 1) % NSLOT2; };
         auto kphase = [&](int v) { return static_cast<uint32_t>(((2 * v) / NSLOT2) & 1); };
         auto vphase = [&](int v) { return static_cast<uint32_t>(((2 * v + 1) / NSLOT2) & 1); };
+        // The issuing thread waits on each tcgen05.mma before it can issue the next one, so any
+        // arithmetic between two MMAs of a group adds to the group's time (it halved the tensor
+        // rate here). Descriptors are therefore formed once, and the eight K-steps of a group
+        // only add constants to the start-address field (addresses stay below 2^18, so the
+        // field never carries into the next one).
+        const uint64_t dqa = k_desc(qbase, 0), dqb = k_desc(qbase + Q_BYTES, 0);
+        const uint64_t dk0 = k_desc(slots, 0), dv0 = v_desc(slots, 0);
         auto qk = [&](int x, int v) {
-          const uint32_t ks = slots + kslot(v) * SLOT_BYTES;
-          const uint32_t qs = qbase + x * Q_BYTES;
+          const uint64_t a0 = x == 0 ? dqa : dqb;
+          const uint64_t b0 = dk0 + static_cast<uint64_t>(kslot(v) * (SLOT_BYTES >> 4));
           const uint32_t d = tmem + (x == 0 ? COL_SA : COL_SB);
-#pragma unroll 1
-          for (int kk = 0; kk < 8; ++kk) mma_ss(d, k_desc(qs, kk), k_desc(ks, kk), IDESC_QK, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t step = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
+            mma_ss(d, a0 + step, b0 + step, IDESC_QK, kk > 0);
+          }
           mma_commit(&s_full[x]);
         };
         auto pv = [&](int x, int v) {
-          const uint32_t vs = slots + vslot(v) * SLOT_BYTES;
+          const uint64_t b0 = dv0 + static_cast<uint64_t>(vslot(v) * (SLOT_BYTES >> 4));
           const uint32_t p_col = tmem + (x == 0 ? COL_SA : COL_SB);
           const uint32_t o_col = tmem + (x == 0 ? COL_OA : COL_OB);
-#pragma unroll 1
-          for (int kk = 0; kk < 8; ++kk) mma_ts(o_col, p_col + kk * 8, v_desc(vs, kk), IDESC_PV, (v > 0) || kk > 0);
+          const uint32_t acc0 = v > 0;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(o_col, p_col + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), IDESC_PV, kk > 0 ? 1u : acc0);
           mma_commit(&o_done[x]);
         };
         // visit 0: S_A, S_B
@@ -309,7 +321,7 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
       }
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;");
     // ------------------------------------------------------------ softmax warps: 0..3 tile A, 4..7 tile B
     const int x = warp >> 2;        // tile
     const int quad = warp & 3;      // TMEM lane quadrant this warp may access
