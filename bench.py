@@ -32,6 +32,35 @@ METRIC = "bifocal prefill TFLOP/s at 128K (frac of BF16 peak); decode µs/step v
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel,
+# from one single-pass ncu capture of a full-size launch (the command is in the profile named
+# below), keyed by the SHA-256 of the kernel's sources at capture time: when the sources no
+# longer match, the kernel has changed since the counters were taken and traffic is null.
+TRAFFIC = {
+    "prefill_attention": {
+        "bytes_per_launch": 48.33e9 + 1.08e9,
+        "sources": ["common.cuh", "prefill_tc.cuh", "prefill_tc2.cuh"],
+        "sha256": "9c2162b6d081b78c78933acf6ffa96faf69194a1baf3b969543d13453d84af70",
+        "profile": "profiles/attn_tc2_traffic_L131072.md",
+    },
+}
+
+
+def measured_traffic(name):
+    import hashlib
+    t = TRAFFIC.get(name)
+    if t is None:
+        return None
+    h = hashlib.sha256()
+    try:
+        for f in t["sources"]:
+            with open(os.path.join(ROOT, "rope_context_extension_bifocal_b200", "csrc", f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    return t["bytes_per_launch"] if h.hexdigest() == t["sha256"] else None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -285,7 +314,8 @@ def run_ours(args):
     attn_tflops = flops / (attn_ms / 1e3) / 1e12
     peak_t = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     roofline = {"bound": "tensor", "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
-                "frac": attn_tflops / peak_t, "traffic": None, "kernel": "bifocal attention (prefill)",
+                "frac": attn_tflops / peak_t, "traffic": measured_traffic("prefill_attention"),
+                "traffic_unit": "bytes per launch (DRAM read + write, ncu)", "kernel": "bifocal attention (prefill)",
                 "peak_kind": f"{peak_kind} bf16 dense burst", "kernel_ms": attn_ms, "rope_pass_ms": rope_ms}
 
     # ---- plain comparator (same shapes, original RoPE only)

@@ -452,12 +452,11 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
   const int nparts = 2 * n_split;
   const int hq = p->hq;
   bf16* o16 = static_cast<bf16*>(out);
+  const dim3 cblock(32 * bf::COMBINE_WARPS);
   if (D == 128)
-    e = launch_pdl(bf::decode_combine_kernel<128>, dim3(p->hq), dim3(128 * bf::COMBINE_GROUPS), 0, st, po, pml, nparts,
-                   hq, o16, lse);
+    e = launch_pdl(bf::decode_combine_kernel<128>, dim3(p->hq, 128 / 32), cblock, 0, st, po, pml, nparts, hq, o16, lse);
   else
-    e = launch_pdl(bf::decode_combine_kernel<64>, dim3(p->hq), dim3(64 * bf::COMBINE_GROUPS), 0, st, po, pml, nparts,
-                   hq, o16, lse);
+    e = launch_pdl(bf::decode_combine_kernel<64>, dim3(p->hq, 64 / 32), cblock, 0, st, po, pml, nparts, hq, o16, lse);
   return e == cudaSuccess ? BF_OK : BF_ERR_CUDA;
 }
 

@@ -350,55 +350,57 @@ constexpr int decode_threads() {
   return (2 * dec::HPC + 3) * 32;  // consumers, TMA warp, two table warps
 }
 
-// Log-sum-exp merge of the split partials: one CTA per query head. The global max comes
-// from a warp-cooperative reduction over the partial maxima; then COMBINE_GROUPS groups of
-// D threads each sum a strided share of the partials for their d, and shared memory adds
-// the groups.
-constexpr int COMBINE_GROUPS = 4;
+// Log-sum-exp merge of the split partials. CTA (h, dq) merges query head h for the 32
+// dimensions 32dq .. 32dq+31, so D/32 CTAs share a head and the grid spreads over the SMs
+// (the merge reads every partial once and is latency-bound, not bandwidth-bound). The
+// global max comes from a block reduction over the partial maxima; then each warp sums a
+// strided share of the partials, one lane per dimension, and shared memory adds the warps.
+constexpr int COMBINE_WARPS = 8;
 
 template <int D>
-__global__ void __launch_bounds__(D * COMBINE_GROUPS) decode_combine_kernel(
+__global__ void __launch_bounds__(32 * COMBINE_WARPS) decode_combine_kernel(
     const float* __restrict__ part_o, const float* __restrict__ part_ml, int n_split, int hq,
     __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
-  __shared__ float red_acc[COMBINE_GROUPS][D];
-  __shared__ float red_l[COMBINE_GROUPS];
-  __shared__ float warp_max[D * COMBINE_GROUPS / 32];
+  __shared__ float red_acc[COMBINE_WARPS][32];
+  __shared__ float red_l[COMBINE_WARPS];
+  __shared__ float warp_max[COMBINE_WARPS];
   pdl_wait();  // the partials of the previous kernel are complete and visible
-  const int h = blockIdx.x, tid = threadIdx.x;
-  const int d = tid % D, grp = tid / D;
-  const int lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.x, d = 32 * blockIdx.y + (threadIdx.x & 31);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // global max of the partial maxima
   float M = -INFINITY;
-  for (int s = tid; s < n_split; s += D * COMBINE_GROUPS) M = fmaxf(M, part_ml[(static_cast<long long>(s) * hq + h) * 2]);
+  for (int s = threadIdx.x; s < n_split; s += 32 * COMBINE_WARPS)
+    M = fmaxf(M, part_ml[(static_cast<long long>(s) * hq + h) * 2]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   if (lane == 0) warp_max[warp] = M;
   __syncthreads();
   M = -INFINITY;
 #pragma unroll
-  for (int w = 0; w < D * COMBINE_GROUPS / 32; ++w) M = fmaxf(M, warp_max[w]);
+  for (int w = 0; w < COMBINE_WARPS; ++w) M = fmaxf(M, warp_max[w]);
   const float ref = (M == -INFINITY) ? 0.f : M;
-  // this group's share of the partials
+  // this warp's share of the partials
   float acc = 0.f, lsum = 0.f;
 #pragma unroll 4
-  for (int s = grp; s < n_split; s += COMBINE_GROUPS) {
+  for (int s = warp; s < n_split; s += COMBINE_WARPS) {
     const long long row = static_cast<long long>(s) * hq + h;
-    const float w = exp2f(part_ml[row * 2] - ref);
-    lsum += w * part_ml[row * 2 + 1];
+    const float2 ml = *reinterpret_cast<const float2*>(part_ml + row * 2);
+    const float w = fast_exp2(ml.x - ref);
+    lsum += w * ml.y;
     acc += w * part_o[row * D + d];
   }
-  red_acc[grp][d] = acc;
-  if (d == 0) red_l[grp] = lsum;
+  red_acc[warp][lane] = acc;
+  if (lane == 0) red_l[warp] = lsum;
   __syncthreads();
-  if (grp == 0) {
+  if (warp == 0) {
     float a = 0.f, l = 0.f;
 #pragma unroll
-    for (int g = 0; g < COMBINE_GROUPS; ++g) {
-      a += red_acc[g][d];
-      l += red_l[g];
+    for (int w = 0; w < COMBINE_WARPS; ++w) {
+      a += red_acc[w][lane];
+      l += red_l[w];
     }
     out[h * D + d] = __float2bfloat16(a / l);
-    if (lse && d == 0) lse[h] = (M + log2f(l)) * 0.69314718055994530942f;
+    if (lse && blockIdx.y == 0 && lane == 0) lse[h] = (M + __log2f(l)) * 0.69314718055994530942f;
   }
 }
 

@@ -245,8 +245,12 @@ __global__ void __launch_bounds__(tc::NTHREADS, 1) attn_tc_kernel(const __grid_c
           const uint32_t s_col = tmem + COL_S + (v & 1) * 128;
           const uint32_t q_col = tmem + (lng ? COL_QL : COL_QO);
           const uint32_t kslot = slots + ks * SLOT_BYTES;
+          // descriptors formed once per group: tcgen05.mma issue waits on the previous MMA, so
+          // arithmetic between the K-steps would stretch the group
+          const uint64_t kd0 = k_desc(kslot, 0);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) mma_ts(s_col, q_col + kk * 8, k_desc(kslot, kk), IDESC_QK, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(s_col, q_col + kk * 8, kd0 + (((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4), IDESC_QK, kk > 0);
           mma_commit(&s_full[v & 1]);
           mma_commit(&empty[ks]);
           // O += P(v-1) V(v-1)
@@ -259,9 +263,11 @@ __global__ void __launch_bounds__(tc::NTHREADS, 1) attn_tc_kernel(const __grid_c
             fence_after();
             const uint32_t p_col = tmem + COL_S + ((v - 1) & 1) * 128;
             const uint32_t vslot = slots + prev_vslot * SLOT_BYTES;
+            const uint64_t vd0 = v_desc(vslot, 0);
+            const uint32_t acc0 = v - 1 > 0;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_ts(tmem + COL_O, p_col + kk * 8, v_desc(vslot, kk), IDESC_PV, (v - 1 > 0) || kk > 0);
+              mma_ts(tmem + COL_O, p_col + kk * 8, vd0 + kk * (2048 >> 4), IDESC_PV, kk > 0 ? 1u : acc0);
             mma_commit(&empty[prev_vslot]);
             mma_commit(&o_done);
           }
@@ -275,9 +281,11 @@ __global__ void __launch_bounds__(tc::NTHREADS, 1) attn_tc_kernel(const __grid_c
           fence_after();
           const uint32_t p_col = tmem + COL_S + ((v - 1) & 1) * 128;
           const uint32_t vslot = slots + prev_vslot * SLOT_BYTES;
+          const uint64_t vd0 = v_desc(vslot, 0);
+          const uint32_t acc0 = v - 1 > 0;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + COL_O, p_col + kk * 8, v_desc(vslot, kk), IDESC_PV, (v - 1 > 0) || kk > 0);
+            mma_ts(tmem + COL_O, p_col + kk * 8, vd0 + kk * (2048 >> 4), IDESC_PV, kk > 0 ? 1u : acc0);
           mma_commit(&empty[prev_vslot]);
           mma_commit(&o_done);
         }

@@ -50,6 +50,8 @@ EDGE = [
     (600, 4, 2, 128, 100, 600, si.POS_ALIAS),     # G == 1
     (1100, 4, 2, 128, 300, 220, si.POS_ALIAS),    # G == 5
     (1100, 4, 2, 128, 300, 367, si.FREQ_INTERP),  # G == 3
+    (1000, 3, 1, 128, 63, 256, si.POS_ALIAS),     # odd GQA group (3): single-tile tcgen05 kernel
+    (600, 2, 2, 128, 100, 150, si.FREQ_INTERP),   # MHA (group 1): single-tile tcgen05 kernel
 ]
 
 
