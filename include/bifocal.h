@@ -133,6 +133,31 @@ BF_API bf_status_t rope_causal_prefill(const void* q, const void* k, const void*
                                 const bf_params_t* p, void* out, float* lse, void* kcache_out, void* vcache_out,
                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* Chunked prefill over an existing cache (batch 1): the step between a prefill and decode,
+ * for a long prompt processed in chunks or new tokens appended to a conversation.
+ *   kcache, vcache [cap, hkv, D] bf16: rows 0..P0-1 hold the cached keys under the ORIGINAL
+ *          RoPE and their values (as bifocal_prefill's kcache_out / bifocal_decode write them);
+ *          rows P0..P0+C-1 are written with the chunk's keys R_orig(P0+r) k_r and its values.
+ *   q    [C, hq,  D] raw, dtype: the chunk's queries at positions P0 .. P0+C-1
+ *   k, v [C, hkv, D] raw, dtype
+ *   out  [C, hq,  D] bf16, written;  lse [hq, C] fp32, written (may be NULL)
+ *   P0 >= 0 cached rows, C >= 1 chunk rows, P0 + C <= cap.
+ * G = max(1, ceil((P0 + C) / w_pretrained)), the factor of the length after the chunk, so it
+ * may differ from the G the cached rows were prefilled under ([AF] module 2: the factor follows
+ * the current length). Chunk row i attends to keys 0..i: pairs with i - j < w0 use the original
+ * RoPE, the others the long-range RoPE, a cached key entering the long branch through the
+ * correction rotation R_long(j) R_orig(j)^-1 ([AF] module 3). The result is rows P0..P0+C-1 of
+ * a bifocal prefill of the whole length whose keys 0..P0-1 are the cached ones.
+ *   workspace / ws_bytes: >= bifocal_prefill_chunk_workspace_size(P0, C, p), 256-byte aligned:
+ *   the chunk's query forms and the key forms of all P0 + C rows (fp16).
+ * Errors: as bifocal_prefill; BF_ERR_INVALID also for NULL caches, P0 < 0, C < 1 or
+ * P0 + C > cap; BF_ERR_UNSUPPORTED unless head_dim == 128 and hq / hkv is even (the tcgen05
+ * ping-pong kernel is the only one with a query offset). */
+BF_API size_t bifocal_prefill_chunk_workspace_size(int32_t P0, int32_t C, const bf_params_t* p);
+BF_API bf_status_t bifocal_prefill_chunk(const void* q, const void* k, const void* v, int32_t dtype, int32_t P0,
+                                         int32_t C, const bf_params_t* p, void* kcache, void* vcache, int32_t cap,
+                                         void* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
 /* Bytes of device workspace bifocal_decode / rope_causal_decode need for a cache of up to
  * L_max rows: the split-KV partial results (fp32). Host only. 0 on invalid arguments. */
 BF_API size_t bifocal_decode_workspace_size(int32_t L_max, const bf_params_t* p);

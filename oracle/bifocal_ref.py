@@ -322,3 +322,49 @@ def bifocal_decode_reference(q, kcache, vcache, L: int, w0: int, w_pretrained: i
             out[h] = (e @ vc[:, kvh]) / e.sum()
             lse[h] = m + math.log(e.sum())
     return out, lse
+
+
+def bifocal_chunk_reference(q, kcache, vcache, P0: int, w0: int, w_pretrained: int, theta: float,
+                            mode: str = FREQ_INTERP, scale: Optional[float] = None,
+                            rows: Optional[Sequence[int]] = None, G: Optional[int] = None):
+    """Chunked prefill over a cache: chunk rows at positions P0 .. P0+C-1 against cache rows 0..L-1.
+
+    q [C, Hq, D] raw chunk queries. kcache [>=L, Hkv, D] (L = P0 + C) holds every key rotated
+    by the original RoPE at its own position - rows 0..P0-1 the cached ones, rows P0.. the
+    chunk's own - and vcache the values. G comes from L, the length after the chunk (the
+    factor follows the current length: ai-feeds summary, 方法 key module 2). Row i attends
+    to keys j <= i. A local key (i - j < w0) scores <R(i omega) q_i, kc_j>; a long-range key is
+    taken back to its raw value with R(-j omega) and rotated by the long-range RoPE of j,
+    against the long-range RoPE of i (the rotation applied to cached keys, key module 3).
+    Returns out [n, Hq, D] and lse [Hq, n] for chunk rows ``rows`` (all C when None).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    C, hq, D = q.shape
+    L = P0 + C
+    kc = np.asarray(kcache[:L], dtype=np.float64)
+    vc = np.asarray(vcache[:L], dtype=np.float64)
+    hkv = kc.shape[1]
+    g = hq // hkv
+    G = dynamic_factor(L, w_pretrained) if G is None else int(G)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    omega = rope_omega(D, theta)
+    rows = np.arange(C, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    pos = np.arange(L, dtype=np.int64)
+    lp, lw = long_branch_rope(pos, omega, G, mode)
+    out = np.empty((len(rows), hq, D))
+    lse = np.empty((hq, len(rows)))
+    for kvh in range(hkv):
+        raw = cached_key_to_raw(kc[:, kvh], pos, omega)
+        k_long = rope_rotate(raw, lp, lw)
+        for h in (hh for hh in range(hq) if kv_head_for(hh, g) == kvh):
+            for n, r in enumerate(rows):
+                i = P0 + int(r)
+                qo = rope_rotate(q[r, h][None], np.array([i]), omega)[0]
+                ql = rope_rotate(q[r, h][None], lp[i:i + 1], lw)[0]
+                s = scale * np.where(i - pos < w0, kc[:, kvh] @ qo, k_long @ ql)
+                s = np.where(pos > i, -np.inf, s)
+                m = s.max()
+                e = np.exp(s - m)
+                out[n, h] = (e @ vc[:, kvh]) / e.sum()
+                lse[h, n] = m + math.log(e.sum())
+    return out, lse

@@ -72,6 +72,10 @@ def _lib() -> ctypes.CDLL:
         L.bifocal_prefill_rope.restype = i32
         L.bifocal_prefill_attention.argtypes = [vp, i32, i32, i32, pp, vp, vp, vp, sz, vp]
         L.bifocal_prefill_attention.restype = i32
+        L.bifocal_prefill_chunk_workspace_size.argtypes = [i32, i32, pp]
+        L.bifocal_prefill_chunk_workspace_size.restype = sz
+        L.bifocal_prefill_chunk.argtypes = [vp, vp, vp, i32, i32, i32, pp, vp, vp, i32, vp, vp, vp, sz, vp]
+        L.bifocal_prefill_chunk.restype = i32
         dec = [vp, vp, vp, vp, vp, i32, i32, pp, vp, vp, vp, sz, vp]
         for name in ("bifocal_decode", "rope_causal_decode"):
             getattr(L, name).argtypes, getattr(L, name).restype = dec, i32
@@ -203,6 +207,30 @@ def rope_causal_prefill(q, k, v, *, theta: float, scale: Optional[float] = None,
     """Plain causal attention under the original RoPE (the comparator)."""
     p = make_params(q.shape[2], k.shape[2], q.shape[3], 0, 1, theta, FREQ_INTERP, scale, 0)
     return _prefill("rope_causal_prefill", q, k, v, p, want_lse, want_cache, out, workspace, stream)
+
+
+def prefill_chunk_workspace_size(P0: int, C: int, params: Params) -> int:
+    return int(_lib().bifocal_prefill_chunk_workspace_size(int(P0), int(C), ctypes.byref(params)))
+
+
+def bifocal_prefill_chunk(q, k, v, kcache, vcache, P0: int, *, w0: int, w_pretrained: int, theta: float,
+                          mode: str = FREQ_INTERP, scale: Optional[float] = None, flags: int = 0,
+                          want_lse: bool = True, out=None, workspace=None, stream=None):
+    """Chunked prefill over a cache (batch 1). q [C, Hq, D], k / v [C, Hkv, D] raw (bf16 or fp32) at
+    positions P0..P0+C-1; kcache / vcache [cap, Hkv, D] bf16 hold P0 cached rows (original-RoPE keys)
+    and receive the chunk's rows. Returns (out [C, Hq, D] bf16, lse [Hq, C] fp32 or None)."""
+    import torch
+    C, hq, D = q.shape
+    p = make_params(hq, k.shape[1], D, w0, w_pretrained, theta, mode, scale, flags)
+    out = torch.empty(C, hq, D, dtype=torch.bfloat16, device=q.device) if out is None else out
+    lse = torch.empty(hq, C, dtype=torch.float32, device=q.device) if want_lse else None
+    need = prefill_chunk_workspace_size(P0, C, p)
+    ws = _workspace(need, q.device) if workspace is None else workspace
+    st = _lib().bifocal_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), int(P0), int(C), ctypes.byref(p),
+                                      _ptr(kcache), _ptr(vcache), kcache.shape[0], _ptr(out), _ptr(lse), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "bifocal_prefill_chunk")
+    return out, lse
 
 
 def _decode(fn_name, q, k_new, v_new, kcache, vcache, L, params, want_lse, out, workspace, stream):

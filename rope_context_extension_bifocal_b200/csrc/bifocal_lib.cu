@@ -218,6 +218,9 @@ bf_status_t prefill_rope_impl(bool bifocal_api, const void* q, const void* k, co
   pa.v = v;
   pa.batch = batch;
   pa.L = L;
+  pa.pos0 = 0;
+  pa.Lk = L;
+  pa.Lc = L;
   pa.hq = p->hq;
   pa.hkv = p->hkv;
   pa.G = plan.G;
@@ -295,6 +298,8 @@ bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtyp
     ta.hkv = p->hkv;
     ta.batch = batch;
     ta.w0 = aa.w0;
+    ta.q_off = 0;
+    ta.Lq = L;
     ta.scale_log2 = aa.scale_log2;
     constexpr int smem = bf::attn_tc2_smem_bytes();
     const long long n_cta = static_cast<long long>((L + bf::tc::BM - 1) / bf::tc::BM) * (p->hq / 2) * batch;
@@ -335,6 +340,126 @@ bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtyp
     e = plan.bif ? launch_attn_mma<128, true>(aa, batch, st) : launch_attn_mma<128, false>(aa, batch, st);
   } else {
     e = plan.bif ? launch_attn_mma<64, true>(aa, batch, st) : launch_attn_mma<64, false>(aa, batch, st);
+  }
+  return e == cudaSuccess ? BF_OK : BF_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ chunked prefill
+struct ChunkLayout {
+  size_t qo, ql, ko, kl, total;
+};
+
+ChunkLayout chunk_layout(int P0, int C, const bf_params_t* p) {
+  ChunkLayout w{};
+  const size_t qbytes = align256(static_cast<size_t>(C) * p->hq * p->head_dim * 2);
+  const size_t kbytes = align256((static_cast<size_t>(P0) + C) * p->hkv * p->head_dim * 2);
+  w.qo = 0;
+  w.ql = w.qo + qbytes;
+  w.ko = w.ql + qbytes;
+  w.kl = w.ko + kbytes;
+  w.total = w.kl + kbytes;
+  return w;
+}
+
+bf_status_t chunk_impl(const void* q, const void* k, const void* v, int32_t dtype, int32_t P0, int32_t C,
+                       const bf_params_t* p, void* kcache, void* vcache, int32_t cap, void* out, float* lse,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  // validate everything before the first launch
+  bf_status_t s = check_params(p, true);
+  if (s != BF_OK) return s;
+  if (!q || !k || !v || !out || !kcache || !vcache) return BF_ERR_INVALID;
+  if (P0 < 0 || C < 1 || cap < 1 || static_cast<int64_t>(P0) + C > cap) return BF_ERR_INVALID;
+  if (dtype != BF_DTYPE_BF16 && dtype != BF_DTYPE_FP32) return BF_ERR_UNSUPPORTED;
+  const int D = p->head_dim, g = p->hq / p->hkv;
+  if (D != 128 || p->hq % 2 || g % 2 || (p->flags & BF_FLAG_MMA_SYNC)) return BF_ERR_UNSUPPORTED;
+  const size_t align_in = dtype == BF_DTYPE_FP32 ? 32 : 16;
+  if (!aligned(q, align_in) || !aligned(k, align_in) || !aligned(v, align_in) || !aligned(kcache, 16) ||
+      !aligned(vcache, 16) || !aligned(out, 16) || (lse && !aligned(lse, 4)))
+    return BF_ERR_INVALID;
+  const int L = P0 + C;
+  const ChunkLayout lay = chunk_layout(P0, C, p);
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < lay.total) return BF_ERR_WORKSPACE;
+  const int G = factor(L, p->w_pretrained);
+  const bool bif = (p->flags & BF_FLAG_FORCE_BIFOCAL) || (G > 1 && p->w0 < L);
+  const Rope rope = make_rope(p->rope_theta, D, G);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  __half* Qo = reinterpret_cast<__half*>(ws + lay.qo);
+  __half* Ql = reinterpret_cast<__half*>(ws + lay.ql);
+  __half* Ko = reinterpret_cast<__half*>(ws + lay.ko);
+  __half* Kl = reinterpret_cast<__half*>(ws + lay.kl);
+
+  // 1. cached keys 0..P0-1 -> Ko (fp16 copy) and Kl (correction rotation)
+  if (P0 > 0) {
+    bf::RephaseArgs ra{};
+    ra.kcache = static_cast<const bf16*>(kcache);
+    ra.P0 = P0;
+    ra.hkv = p->hkv;
+    ra.Lk = L;
+    ra.G = G;
+    ra.mode = p->mode;
+    ra.need_long = bif ? 1 : 0;
+    ra.Ko = Ko;
+    ra.Kl = Kl;
+    std::memcpy(ra.omega, rope.omega, sizeof(ra.omega));
+    std::memcpy(ra.omega_corr, rope.omega_corr, sizeof(ra.omega_corr));
+    bf::cache_rephase_kernel<128><<<static_cast<unsigned>((P0 + 7) / 8), 256, 0, st>>>(ra);
+    if (cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
+  }
+  // 2. the chunk: RoPE forms of q and k at positions P0.., key rows P0.., cache rows P0..
+  bf::PrepassArgs pa{};
+  pa.q = q;
+  pa.k = k;
+  pa.v = v;
+  pa.batch = 1;
+  pa.L = C;
+  pa.pos0 = P0;
+  pa.Lk = L;
+  pa.Lc = cap;
+  pa.hq = p->hq;
+  pa.hkv = p->hkv;
+  pa.G = G;
+  pa.mode = p->mode;
+  pa.need_long = bif ? 1 : 0;
+  pa.Qo = Qo;
+  pa.Ql = Ql;
+  pa.Ko = Ko;
+  pa.Kl = Kl;
+  pa.Vb = nullptr;
+  pa.kcache = static_cast<bf16*>(kcache);
+  pa.vcache = static_cast<bf16*>(vcache);
+  std::memcpy(pa.omega, rope.omega, sizeof(pa.omega));
+  std::memcpy(pa.omega_long, rope.omega_long, sizeof(pa.omega_long));
+  const dim3 pgrid(static_cast<unsigned>((C + 7) / 8));
+  if (dtype == BF_DTYPE_BF16)
+    bf::rope_prepass_kernel<bf16, 128><<<pgrid, 256, 0, st>>>(pa);
+  else
+    bf::rope_prepass_kernel<float, 128><<<pgrid, 256, 0, st>>>(pa);
+  if (cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
+  // 3. attention of the C query rows (absolute positions P0..) over keys 0..L-1; V is the cache
+  bf::Tc2Args ta;
+  std::memset(&ta, 0, sizeof(ta));
+  if (!make_k_map(&ta.qo_map, Qo, C, p->hq) || !make_k_map(&ta.ql_map, Ql, C, p->hq) ||
+      !make_k_map(&ta.ko_map, Ko, L, p->hkv) || !make_k_map(&ta.kl_map, Kl, L, p->hkv) ||
+      !make_v_map(&ta.v_map, vcache, L, p->hkv, 1))
+    return BF_ERR_CUDA;
+  ta.out = static_cast<bf16*>(out);
+  ta.lse = lse;
+  ta.L = L;
+  ta.hq = p->hq;
+  ta.hkv = p->hkv;
+  ta.batch = 1;
+  ta.w0 = bif ? p->w0 : L;
+  ta.q_off = P0;
+  ta.Lq = C;
+  ta.scale_log2 = scale_log2(p);
+  constexpr int smem = bf::attn_tc2_smem_bytes();
+  const long long n_cta = static_cast<long long>((C + bf::tc::BM - 1) / bf::tc::BM) * (p->hq / 2);
+  auto kern = bif ? bf::attn_tc2_kernel<true> : bf::attn_tc2_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) {
+    kern<<<static_cast<unsigned>(n_cta), bf::tc2::NTHREADS2, smem, st>>>(ta);
+    e = cudaGetLastError();
   }
   return e == cudaSuccess ? BF_OK : BF_ERR_CUDA;
 }
@@ -503,6 +628,17 @@ bf_status_t bifocal_prefill(const void* q, const void* k, const void* v, int32_t
                             void* workspace, size_t ws_bytes, void* stream) {
   return prefill_impl(true, q, k, v, dtype, batch, L, p, out, lse, kcache_out, vcache_out, workspace, ws_bytes,
                       stream);
+}
+
+size_t bifocal_prefill_chunk_workspace_size(int32_t P0, int32_t C, const bf_params_t* p) {
+  if (check_params(p, true) != BF_OK || P0 < 0 || C < 1 || static_cast<int64_t>(P0) + C > 0x7fffffff) return 0;
+  return chunk_layout(P0, C, p).total;
+}
+
+bf_status_t bifocal_prefill_chunk(const void* q, const void* k, const void* v, int32_t dtype, int32_t P0, int32_t C,
+                                  const bf_params_t* p, void* kcache, void* vcache, int32_t cap, void* out, float* lse,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+  return chunk_impl(q, k, v, dtype, P0, C, p, kcache, vcache, cap, out, lse, workspace, ws_bytes, stream);
 }
 
 bf_status_t bifocal_prefill_rope(const void* q, const void* k, const void* v, int32_t dtype, int32_t batch,

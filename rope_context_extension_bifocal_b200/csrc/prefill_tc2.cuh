@@ -108,9 +108,12 @@ struct Tc2Args {
   CUtensorMap ko_map;  // fp16 [b*hkv][L][128]
   CUtensorMap kl_map;
   CUtensorMap v_map;   // bf16 [b][L][hkv][128], box (64, 1, 128, 1)
-  __nv_bfloat16* out;  // [b, L, hq, 128]
-  float* lse;          // [b, hq, L] or null
+  __nv_bfloat16* out;  // [b, Lq, hq, 128]
+  float* lse;          // [b, hq, Lq] or null
   int L, hq, hkv, batch, w0;
+  // query rows: Lq rows at absolute positions q_off .. q_off + Lq - 1 (a full prefill has
+  // q_off = 0 and Lq = L; a chunk over a cache has q_off = the cached length); keys 0 .. L-1
+  int q_off, Lq;
   float scale_log2;
 };
 
@@ -123,7 +126,7 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
   __shared__ int s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_qt = (a.L + BM - 1) / BM;
+  const int n_qt = (a.Lq + BM - 1) / BM;
   const int pairs = a.hq / 2;
   const int per_tile = pairs * a.batch;
   const int qt = n_qt - 1 - static_cast<int>(blockIdx.x) / per_tile;  // heaviest first
@@ -131,8 +134,8 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
   const int hp = rem % pairs, b = rem / pairs;
   const int h0 = 2 * hp;  // heads h0 (tile A) and h0 + 1 (tile B), same kv head
   const int kvh = h0 / (a.hq / a.hkv);
-  const int i0 = qt * BM;
-  const int n_kt = (min(i0 + BM, a.L) + BN - 1) / BN;
+  const int i0 = a.q_off + qt * BM;  // absolute position of the tile's first query row
+  const int n_kt = (min(i0 + BM, a.q_off + a.Lq) + BN - 1) / BN;
   const Schedule sch = make_schedule<BIFOCAL>(i0, n_kt, a.w0);
   const int nv = sch.total();
   const bool has_long = sch.n_long() > 0;
@@ -190,8 +193,8 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
           mbar_arrive_expect_tx(&q_full, 2 * Q_BYTES);
           for (int x = 0; x < 2; ++x) {
             uint8_t* dst = smem + x * Q_BYTES;
-            tma_load_3d(dst, m, &q_full, 0, i0, qrow + x);
-            tma_load_3d(dst + HALF_BYTES, m, &q_full, 64, i0, qrow + x);
+            tma_load_3d(dst, m, &q_full, 0, qt * BM, qrow + x);
+            tma_load_3d(dst + HALF_BYTES, m, &q_full, 64, qt * BM, qrow + x);
           }
         };
         load_q(has_long ? &a.ql_map : &a.qo_map);
@@ -470,13 +473,14 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
     if (ok && nv > 0 && __all_sync(0xffffffffu, mbar_wait_abortable(&o_done[x], (nv - 1) & 1, 32, &s_abort))) {
       fence_after();
       const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      __nv_bfloat16* orow = a.out + ((static_cast<long long>(b) * a.L + i) * a.hq + h) * D;
+      const int rel = i - a.q_off;  // row of this query in out / lse
+      __nv_bfloat16* orow = a.out + ((static_cast<long long>(b) * a.Lq + rel) * a.hq + h) * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < 128; c0 += 32) {
         float ov[32];
         tmem_ld32(o_col + c0, ov);
         wait_ld();
-        if (i < a.L) {
+        if (rel < a.Lq) {
 #pragma unroll
           for (int u = 0; u < 32; u += 8) {
             uint4 w;
@@ -488,8 +492,8 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
           }
         }
       }
-      if (a.lse && i < a.L)
-        a.lse[(static_cast<long long>(b) * a.hq + h) * a.L + i] = (m_ref + __log2f(l_sum)) * 0.69314718055994530942f;
+      if (a.lse && rel < a.Lq)
+        a.lse[(static_cast<long long>(b) * a.hq + h) * a.Lq + rel] = (m_ref + __log2f(l_sum)) * 0.69314718055994530942f;
     }
   }
 

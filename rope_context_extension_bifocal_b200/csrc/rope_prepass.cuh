@@ -11,7 +11,16 @@
 // interpolation) or floor(p / G) * omega_k (position aliasing) - the two long-range
 // forms named by the ablation of the ai-feeds summary of Jet-Long (实验, key findings).
 // Ko is also the decode cache (keys under the original RoPE) and is written to the
-// caller's kcache in [b, L, hkv, D] when asked. fp32 inputs are rounded to bf16 here.
+// caller's kcache in [b, Lc, hkv, D] when asked. fp32 inputs are rounded to bf16 here.
+// A chunk over an existing cache passes its first absolute position in pos0: the angles,
+// the key rows and the cache rows are those of positions pos0 .. pos0 + L - 1.
+//
+// cache_rephase_kernel prepares the cached part of a chunked prefill: the cache holds
+// keys under the original RoPE (bf16), so Ko is their fp16 copy (exact: a bf16 value
+// of normal magnitude has 8 significant bits, fp16 11), and Kl re-phases them by the
+// correction rotation R_long(j) R_orig(j)^-1 - angle j * omega_k * (1/G - 1) under
+// frequency interpolation, (floor(j/G) - j) * omega_k under position aliasing (the
+// rotation applied to cached keys in the ai-feeds summary of Jet-Long, 方法 key module 3).
 #pragma once
 #include "common.cuh"
 
@@ -21,7 +30,10 @@ struct PrepassArgs {
   const void* q;
   const void* k;
   const void* v;
-  int batch, L, hq, hkv;
+  int batch, L, hq, hkv;  // L rows of q, k, v per batch (a full prompt, or a chunk)
+  int pos0;               // absolute position of row 0 (0, or the cached length for a chunk)
+  int Lk;                 // rows of Ko / Kl per (batch, kv head): pos0 + L for a chunk
+  int Lc;                 // rows of kcache / vcache per batch
   int G;
   int mode;       // 0 = frequency interpolation, 1 = position aliasing
   int need_long;  // write Ql / Kl
@@ -91,7 +103,8 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
   const long long gpos = static_cast<long long>(blockIdx.x) * 8 + warp;
   if (gpos >= static_cast<long long>(a.batch) * a.L) return;
   const int b = static_cast<int>(gpos / a.L);
-  const int p = static_cast<int>(gpos % a.L);
+  const int r_in = static_cast<int>(gpos % a.L);  // row of the input
+  const int p = a.pos0 + r_in;                     // absolute position
   const int grp = lane >> 3, l8 = lane & 7;
   if (l8 >= LANES_PER_ROW) return;
   const int k0 = l8 * NPAIR;  // first pair index this lane owns
@@ -120,7 +133,7 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
     const bool is_q = r < a.hq;
     const int h = is_q ? r : r - a.hq;
     const int H = is_q ? a.hq : a.hkv;
-    const Tin* src = (is_q ? qb : kb) + ((static_cast<long long>(b) * a.L + p) * H + h) * D;
+    const Tin* src = (is_q ? qb : kb) + ((static_cast<long long>(b) * a.L + r_in) * H + h) * D;
     Vec8<Tin> x1, x2;
     x1.load(src + k0);
     x2.load(src + P + k0);
@@ -133,7 +146,9 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
       yl1[i] = u * cl[i] - w * sl[i];
       yl2[i] = w * cl[i] + u * sl[i];
     }
-    const long long hm = ((static_cast<long long>(b) * H + h) * a.L + p) * D;  // head-major row
+    // head-major rows: Q has the input's L rows, K the Lk rows of keys 0 .. Lk-1
+    const long long hm = is_q ? ((static_cast<long long>(b) * H + h) * a.L + r_in) * D
+                              : ((static_cast<long long>(b) * H + h) * a.Lk + p) * D;
     __half* dst_o = (is_q ? a.Qo : a.Ko) + hm;
     store8_f16(dst_o + k0, yo1);
     store8_f16(dst_o + P + k0, yo2);
@@ -143,7 +158,7 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
       store8_f16(dst_l + P + k0, yl2);
     }
     if (!is_q && a.kcache) {
-      __nv_bfloat16* dc = a.kcache + ((static_cast<long long>(b) * a.L + p) * a.hkv + h) * D;
+      __nv_bfloat16* dc = a.kcache + ((static_cast<long long>(b) * a.Lc + p) * a.hkv + h) * D;
       store8_bf16(dc + k0, yo1);
       store8_bf16(dc + P + k0, yo2);
     }
@@ -151,7 +166,8 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
   // v: bf16 copy for fp32 inputs and / or the caller's vcache
   if (a.Vb || a.vcache) {
     for (int h = grp; h < a.hkv; h += 4) {
-      const long long off = ((static_cast<long long>(b) * a.L + p) * a.hkv + h) * D;
+      const long long off = ((static_cast<long long>(b) * a.L + r_in) * a.hkv + h) * D;
+      const long long coff = ((static_cast<long long>(b) * a.Lc + p) * a.hkv + h) * D;
       Vec8<Tin> x1, x2;
       x1.load(vb + off + k0);
       x2.load(vb + off + P + k0);
@@ -166,9 +182,68 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
         store8_bf16(a.Vb + off + P + k0, y2);
       }
       if (a.vcache) {
-        store8_bf16(a.vcache + off + k0, y1);
-        store8_bf16(a.vcache + off + P + k0, y2);
+        store8_bf16(a.vcache + coff + k0, y1);
+        store8_bf16(a.vcache + coff + P + k0, y2);
       }
+    }
+  }
+}
+
+struct RephaseArgs {
+  const __nv_bfloat16* kcache;  // [Lc, hkv, D], rows 0 .. P0-1 read
+  int P0, hkv, Lk;              // cached rows; kv heads; rows of Ko / Kl per kv head
+  int G, mode, need_long;
+  __half* Ko;                   // [hkv, Lk, D]
+  __half* Kl;
+  double omega[64];
+  double omega_corr[64];        // omega_k * (1/G - 1)
+};
+
+// One warp per cached position, all kv heads; lanes as in rope_prepass_kernel.
+template <int D>
+__global__ void __launch_bounds__(256) cache_rephase_kernel(const __grid_constant__ RephaseArgs a) {
+  constexpr int P = D / 2;
+  constexpr int NPAIR = 8;
+  constexpr int LANES_PER_ROW = P / NPAIR;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long j_ll = static_cast<long long>(blockIdx.x) * 8 + warp;
+  if (j_ll >= a.P0) return;
+  const int j = static_cast<int>(j_ll);
+  const int grp = lane >> 3, l8 = lane & 7;
+  if (l8 >= LANES_PER_ROW) return;
+  const int k0 = l8 * NPAIR;
+  float cc[NPAIR], sc[NPAIR];
+  if (a.need_long) {
+    const double jd = static_cast<double>(j);
+    const double jg = static_cast<double>(j / a.G - j);
+#pragma unroll
+    for (int i = 0; i < NPAIR; ++i)
+      angle_cos_sin(a.mode == 0 ? jd * a.omega_corr[k0 + i] : jg * a.omega[k0 + i], cc[i], sc[i]);
+  }
+  for (int h = grp; h < a.hkv; h += 4) {
+    const __nv_bfloat16* src = a.kcache + (static_cast<long long>(j) * a.hkv + h) * D;
+    Vec8<__nv_bfloat16> x1, x2;
+    x1.load(src + k0);
+    x2.load(src + P + k0);
+    float u[8], w[8];
+#pragma unroll
+    for (int i = 0; i < NPAIR; ++i) {
+      u[i] = x1.get(i);
+      w[i] = x2.get(i);
+    }
+    __half* dst_o = a.Ko + (static_cast<long long>(h) * a.Lk + j) * D;
+    store8_f16(dst_o + k0, u);
+    store8_f16(dst_o + P + k0, w);
+    if (a.need_long) {
+      float y1[8], y2[8];
+#pragma unroll
+      for (int i = 0; i < NPAIR; ++i) {
+        y1[i] = u[i] * cc[i] - w[i] * sc[i];
+        y2[i] = w[i] * cc[i] + u[i] * sc[i];
+      }
+      __half* dst_l = a.Kl + (static_cast<long long>(h) * a.Lk + j) * D;
+      store8_f16(dst_l + k0, y1);
+      store8_f16(dst_l + P + k0, y2);
     }
   }
 }

@@ -129,6 +129,34 @@ def test_decode_validation_before_launch(lib, fn):
     assert call(params(), wsb=16) == 5
 
 
+def test_chunk_workspace_size(lib):
+    p = params()
+    P0, C = 126976, 4096
+    L = P0 + C
+    # fp16 Qo/Ql [C, 32, 128] and Ko/Kl [L, 8, 128]
+    assert bfl.prefill_chunk_workspace_size(P0, C, p) == 2 * (C * 32 * 128 * 2) + 2 * (L * 8 * 128 * 2)
+    assert bfl.prefill_chunk_workspace_size(-1, C, p) == 0
+    assert bfl.prefill_chunk_workspace_size(P0, 0, p) == 0
+
+
+def test_chunk_validation_before_launch(lib):
+    f = lib.bifocal_prefill_chunk
+
+    def call(p, P0=100, C=50, cap=200, kc=FAKE, ws=FAKE, wsb=1 << 30, dtype=0):
+        return f(FAKE, FAKE, FAKE, dtype, P0, C, ctypes.byref(p), kc, FAKE, cap, FAKE, None, ws, wsb, None)
+
+    assert call(params(), kc=None) == 1
+    assert call(params(), P0=-1) == 1
+    assert call(params(), C=0) == 1
+    assert call(params(), P0=190, C=11) == 1       # P0 + C > cap
+    assert call(params(head_dim=64)) == 2           # only the D = 128 ping-pong kernel takes a query offset
+    assert call(params(hq=24, hkv=8)) == 2          # odd GQA group
+    assert call(params(), dtype=4) == 2
+    assert call(params(w0=-1)) == 1
+    assert call(params(), ws=None) == 5
+    assert call(params(), wsb=256) == 5
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     mod = importlib.import_module("rope_context_extension_bifocal_b200")
