@@ -38,9 +38,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # longer match, the kernel has changed since the counters were taken and traffic is null.
 TRAFFIC = {
     "prefill_attention": {
-        "bytes_per_launch": 48.33e9 + 1.08e9,
+        "bytes_per_launch": 60.62e9 + 1.11e9,
         "sources": ["common.cuh", "prefill_tc.cuh", "prefill_tc2.cuh"],
-        "sha256": "9c2162b6d081b78c78933acf6ffa96faf69194a1baf3b969543d13453d84af70",
+        "sha256": "b5d7f2e31ad8806c5666de6ea4e04cfb217ab0415fab212aa6554ff7b5b692fb",
         "profile": "profiles/attn_tc2_traffic_L131072.md",
     },
 }
@@ -389,6 +389,24 @@ def run_ours(args):
                          "FLOPs counted over the chunk's causal pairs"}
         del kc_all, vc_all, wsc, outc
 
+    # ---- sliding-window prefill (the local layers of a hybrid model), window = w0
+    window = None
+    if not args.no_window:
+        pw = bfl.make_params(w.hq, w.hkv, w.head_dim, w.w0, w.w_pretrained, w.theta, w.mode, None, bfl.FLAG_WINDOW)
+
+        def step_window():
+            bfl.bifocal_prefill_rope(q, k, v, pw, ws)
+            bfl.bifocal_prefill_attention(v, pw, ws, out, lse)
+
+        n_win = max(3, args.steps)
+        win_ms = time_loop(step_window, n_win, 1, dist, torch) / n_win
+        Wn = min(w.w0, w.L)
+        pairs = Wn * (Wn + 1) / 2 + (w.L - Wn) * Wn  # causal pairs with i - j < w0
+        win_tflops = 4.0 * w.head_dim * w.hq * pairs / (win_ms / 1e3) / 1e12
+        window = {"workload": f"qwen3_8b_L{w.L}_window{Wn}", "window": Wn, "ms": win_ms, "tflops": win_tflops,
+                  "frac_of_peak": win_tflops / peak_t,
+                  "note": "BF_FLAG_WINDOW prefill (RoPE pass + attention); FLOPs counted over the window's pairs"}
+
     # ---- decode: 200 steps across the G = 4 -> 5 change
     decode = None
     if not args.no_decode:
@@ -423,6 +441,7 @@ def run_ours(args):
         "w0_sweep": sweep,
         "decode": decode,
         "chunked_prefill": chunk,
+        "window_prefill": window,
         "build": bfl.build_info(),
     }
     if dist.rank == 0:
@@ -468,8 +487,14 @@ def run_decode(args, torch, bfl, si, dev, peaks, peak_kind):
         bfl.rope_causal_decode(q, kn, vn, kcache, vcache, w.prefix_len + t + 1, theta=w.theta, out=out,
                                workspace=ws)
 
+    def window(t):  # the local layers of a hybrid model: keys L - w0 .. L - 1 only
+        q, kn, vn = steps[t]
+        bfl.bifocal_decode(q, kn, vn, kcache, vcache, w.prefix_len + t + 1, w0=w.w0, w_pretrained=w.w_pretrained,
+                           theta=w.theta, mode=w.mode, flags=bfl.FLAG_WINDOW, out=out, workspace=ws)
+
     us = session(bif)
     us_plain = session(plain)
+    us_window = session(window)
     gbs = [w.cache_bytes(w.prefix_len + t + 1) / (u * 1e-6) / 1e9 for t, u in enumerate(us)]
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     med = statistics.median(us)
@@ -487,6 +512,9 @@ def run_decode(args, torch, bfl, si, dev, peaks, peak_kind):
                      "peak_kind": f"{peak_kind} HBM copy",
                      "bytes_per_step_at_131072": w.cache_bytes(131072)},
         "gpu_launches": 3 * len(us),
+        "window": {"w0": w.w0, "us_median": statistics.median(us_window),
+                   "bytes_per_step": 4 * w.hkv * w.head_dim * w.w0,
+                   "note": "sliding-window decode (BF_FLAG_WINDOW): reads the last w0 cached tokens"},
     }
 
 
@@ -500,6 +528,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-chunk", action="store_true")
+    ap.add_argument("--no-window", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -71,6 +71,12 @@ typedef enum { BF_DTYPE_BF16 = 0, BF_DTYPE_FP32 = 1 } bf_dtype_t;
 #define BF_FLAG_FORCE_BIFOCAL 1 /* run the two-branch kernel even when G == 1 or w0 >= L (results are equal) */
 #define BF_FLAG_MMA_SYNC 2      /* prefill, D = 128: use the warp-level mma.sync kernel instead of tcgen05
                                    (comparison only; D = 64 always uses it) */
+#define BF_FLAG_WINDOW 4        /* sliding-window attention, the local layers of a hybrid model (Jet-Nemotron,
+                                 * [AF] 影响): keep only pairs with 0 <= i - j < w0, under the original RoPE;
+                                 * the long-range branch is dropped and G plays no part. Taken by
+                                 * bifocal_prefill (+ its two steps), bifocal_prefill_chunk and bifocal_decode;
+                                 * needs w0 >= 1 (BF_ERR_INVALID otherwise) and, for the prefill forms,
+                                 * head_dim 128 with an even GQA group (BF_ERR_UNSUPPORTED otherwise) */
 
 typedef struct {
   int32_t hq;           /* query heads; hq % hkv == 0; query head h reads kv head h / (hq / hkv) */

@@ -368,3 +368,72 @@ def bifocal_chunk_reference(q, kcache, vcache, P0: int, w0: int, w_pretrained: i
                 out[n, h] = (e @ vc[:, kvh]) / e.sum()
                 lse[h, n] = m + math.log(e.sum())
     return out, lse
+
+
+# ----------------------------------------------------------------------------------
+# Sliding-window attention: the local layers of a hybrid model (Jet-Nemotron, named by the
+# ai-feeds summary, 影响 / 局限) keep only the near keys, under the original RoPE
+# ----------------------------------------------------------------------------------
+def sliding_window_attention(q, k, v, window: int, theta: float, scale: Optional[float] = None,
+                             rows: Optional[Sequence[int]] = None):
+    """Causal attention restricted to 0 <= i - j < window, original RoPE, fp64.
+
+    Same layouts as :func:`bifocal_attention`; window >= 1.
+    """
+    q, k, v = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
+    b, L, hq, hkv, D = _check(q, k, v)
+    if window < 1:
+        raise ValueError("window must be >= 1")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    rows = np.arange(L, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    omega = rope_omega(D, theta)
+    g = hq // hkv
+    pos = np.arange(L, dtype=np.int64)
+    dist = rows[:, None] - pos[None, :]
+    keep = (dist >= 0) & (dist < window)
+    out = np.empty((b, len(rows), hq, D))
+    lse = np.empty((b, hq, len(rows)))
+    for bi in range(b):
+        for h in range(hq):
+            kvh = kv_head_for(h, g)
+            kr = rope_rotate(k[bi, :, kvh], pos, omega)
+            qr = rope_rotate(q[bi, rows, h], rows, omega)
+            s = np.where(keep, scale * (qr @ kr.T), -np.inf)
+            o, ls = _softmax_out(s, v[bi, :, kvh])
+            out[bi, :, h] = o
+            lse[bi, h] = ls
+    return out, lse
+
+
+def sliding_window_cached_reference(q, kcache, vcache, P0: int, window: int, theta: float,
+                                    scale: Optional[float] = None, rows: Optional[Sequence[int]] = None):
+    """Sliding-window rows at positions P0 .. P0+C-1 against a cache of original-RoPE keys.
+
+    q [C, Hq, D] raw; kcache / vcache [>= P0 + C, Hkv, D] as stored (row j = R(j omega) k_j).
+    Covers a chunk over a cache and a decode step (C = 1, P0 = L - 1). Row i scores
+    <R(i omega) q_i, kc_j> for 0 <= i - j < window. Returns out [n, Hq, D], lse [Hq, n].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    C, hq, D = q.shape
+    L = P0 + C
+    kc = np.asarray(kcache[:L], dtype=np.float64)
+    vc = np.asarray(vcache[:L], dtype=np.float64)
+    g = hq // kc.shape[1]
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    omega = rope_omega(D, theta)
+    rows = np.arange(C, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    pos = np.arange(L, dtype=np.int64)
+    out = np.empty((len(rows), hq, D))
+    lse = np.empty((hq, len(rows)))
+    for h in range(hq):
+        kvh = kv_head_for(h, g)
+        for n, r in enumerate(rows):
+            i = P0 + int(r)
+            qo = rope_rotate(q[r, h][None], np.array([i]), omega)[0]
+            keep = (i - pos >= 0) & (i - pos < window)
+            s = np.where(keep, scale * (kc[:, kvh] @ qo), -np.inf)
+            m = s.max()
+            e = np.exp(s - m)
+            out[n, h] = (e @ vc[:, kvh]) / e.sum()
+            lse[h, n] = m + math.log(e.sum())
+    return out, lse

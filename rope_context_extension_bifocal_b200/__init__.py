@@ -14,7 +14,7 @@ import os
 from typing import Optional, Tuple
 
 __all__ = [
-    "BifocalError", "FREQ_INTERP", "POS_ALIAS", "FLAG_FORCE_BIFOCAL", "FLAG_MMA_SYNC", "Params", "lib", "lib_path",
+    "BifocalError", "FREQ_INTERP", "POS_ALIAS", "FLAG_FORCE_BIFOCAL", "FLAG_MMA_SYNC", "FLAG_WINDOW", "Params", "lib", "lib_path",
     "bifocal_factor", "bifocal_prefill", "bifocal_prefill_rope", "bifocal_prefill_attention", "rope_causal_prefill", "bifocal_decode", "bifocal_decode_noalloc", "rope_causal_decode",
     "prefill_workspace_size", "decode_workspace_size", "last_device_error", "build_info",
 ]
@@ -24,6 +24,7 @@ POS_ALIAS = "pos_alias"
 _MODES = {FREQ_INTERP: 0, POS_ALIAS: 1}
 FLAG_FORCE_BIFOCAL = 1
 FLAG_MMA_SYNC = 2
+FLAG_WINDOW = 4
 DTYPE_BF16, DTYPE_FP32 = 0, 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))

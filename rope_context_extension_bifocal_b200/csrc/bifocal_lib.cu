@@ -172,11 +172,18 @@ cudaError_t launch_attn_mma(const bf::AttnArgs& a, int batch, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// The tcgen05 ping-pong kernel (two heads of one GQA group per CTA) takes D = 128 and an even group.
+bool tc2_path(const bf_params_t* p) {
+  const int g = p->hq / p->hkv;
+  return p->head_dim == 128 && !(p->flags & BF_FLAG_MMA_SYNC) && p->hq % 2 == 0 && g % 2 == 0;
+}
+
 // What a prefill call resolves before any launch (shared by the one-call form and the
 // two steps, so both make the same choice).
 struct PrefillPlan {
   int D, G;
   bool bif;  // two-branch kernel (else every pair is local: the plain kernel gives the same result)
+  int kind;  // tcgen05 ping-pong kernel: KIND_PLAIN, KIND_BIFOCAL or KIND_WINDOW
   PrefillLayout lay;
   Rope rope;
 };
@@ -187,11 +194,15 @@ bf_status_t plan_prefill(bool bifocal_api, int32_t dtype, int32_t batch, int32_t
   if (s != BF_OK) return s;
   if (batch < 1 || L < 1) return BF_ERR_INVALID;
   if (dtype != BF_DTYPE_BF16 && dtype != BF_DTYPE_FP32) return BF_ERR_UNSUPPORTED;
+  const bool window = bifocal_api && (p->flags & BF_FLAG_WINDOW);
+  if (window && p->w0 < 1) return BF_ERR_INVALID;
+  if (window && !tc2_path(p)) return BF_ERR_UNSUPPORTED;
   plan->lay = prefill_layout(dtype, batch, L, p);
   if (!workspace || !aligned(workspace, 256) || ws_bytes < plan->lay.total) return BF_ERR_WORKSPACE;
   plan->D = p->head_dim;
   plan->G = bifocal_api ? factor(L, p->w_pretrained) : 1;
-  plan->bif = bifocal_api && ((p->flags & BF_FLAG_FORCE_BIFOCAL) || (plan->G > 1 && p->w0 < L));
+  plan->bif = !window && bifocal_api && ((p->flags & BF_FLAG_FORCE_BIFOCAL) || (plan->G > 1 && p->w0 < L));
+  plan->kind = window ? (p->w0 < L ? bf::tc2::KIND_WINDOW : bf::tc2::KIND_PLAIN) : (plan->bif ? bf::tc2::KIND_BIFOCAL : bf::tc2::KIND_PLAIN);
   plan->rope = make_rope(p->rope_theta, plan->D, plan->G);
   return BF_OK;
 }
@@ -279,11 +290,11 @@ bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtyp
   aa.L = L;
   aa.hq = p->hq;
   aa.hkv = p->hkv;
-  aa.w0 = plan.bif ? p->w0 : L;
+  aa.w0 = plan.kind != bf::tc2::KIND_PLAIN ? p->w0 : L;
   aa.scale_log2 = scale_log2(p);
   cudaError_t e;
   const int g = p->hq / p->hkv;
-  if (D == 128 && !(p->flags & BF_FLAG_MMA_SYNC) && p->hq % 2 == 0 && g % 2 == 0) {
+  if (tc2_path(p)) {
     // tcgen05 ping-pong path: two heads of one GQA group per CTA
     bf::Tc2Args ta;
     std::memset(&ta, 0, sizeof(ta));
@@ -304,7 +315,9 @@ bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtyp
     constexpr int smem = bf::attn_tc2_smem_bytes();
     const long long n_cta = static_cast<long long>((L + bf::tc::BM - 1) / bf::tc::BM) * (p->hq / 2) * batch;
     if (n_cta > 0x7fffffffLL) return BF_ERR_UNSUPPORTED;
-    auto kern = plan.bif ? bf::attn_tc2_kernel<true> : bf::attn_tc2_kernel<false>;
+    auto kern = plan.kind == bf::tc2::KIND_BIFOCAL  ? bf::attn_tc2_kernel<bf::tc2::KIND_BIFOCAL>
+                : plan.kind == bf::tc2::KIND_WINDOW ? bf::attn_tc2_kernel<bf::tc2::KIND_WINDOW>
+                                               : bf::attn_tc2_kernel<bf::tc2::KIND_PLAIN>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess) {
       kern<<<static_cast<unsigned>(n_cta), bf::tc2::NTHREADS2, smem, st>>>(ta);
@@ -377,10 +390,13 @@ bf_status_t chunk_impl(const void* q, const void* k, const void* v, int32_t dtyp
       !aligned(vcache, 16) || !aligned(out, 16) || (lse && !aligned(lse, 4)))
     return BF_ERR_INVALID;
   const int L = P0 + C;
+  const bool window = (p->flags & BF_FLAG_WINDOW) != 0;
+  if (window && p->w0 < 1) return BF_ERR_INVALID;
   const ChunkLayout lay = chunk_layout(P0, C, p);
   if (!workspace || !aligned(workspace, 256) || ws_bytes < lay.total) return BF_ERR_WORKSPACE;
   const int G = factor(L, p->w_pretrained);
-  const bool bif = (p->flags & BF_FLAG_FORCE_BIFOCAL) || (G > 1 && p->w0 < L);
+  const bool bif = !window && ((p->flags & BF_FLAG_FORCE_BIFOCAL) || (G > 1 && p->w0 < L));
+  const int kind = window ? (p->w0 < L ? bf::tc2::KIND_WINDOW : bf::tc2::KIND_PLAIN) : (bif ? bf::tc2::KIND_BIFOCAL : bf::tc2::KIND_PLAIN);
   const Rope rope = make_rope(p->rope_theta, D, G);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -389,13 +405,16 @@ bf_status_t chunk_impl(const void* q, const void* k, const void* v, int32_t dtyp
   __half* Ko = reinterpret_cast<__half*>(ws + lay.ko);
   __half* Kl = reinterpret_cast<__half*>(ws + lay.kl);
 
-  // 1. cached keys 0..P0-1 -> Ko (fp16 copy) and Kl (correction rotation)
-  if (P0 > 0) {
+  // 1. cached keys -> Ko (fp16 copy) and Kl (correction rotation). A window reads only the
+  //    cached keys within w0 of the chunk, from the start of their key tile on.
+  const int j_begin = kind == bf::tc2::KIND_WINDOW ? std::max(0, (P0 + 1 - p->w0) / bf::tc::BN * bf::tc::BN) : 0;
+  if (P0 > j_begin) {
     bf::RephaseArgs ra{};
     ra.kcache = static_cast<const bf16*>(kcache);
     ra.P0 = P0;
     ra.hkv = p->hkv;
     ra.Lk = L;
+    ra.j_begin = j_begin;
     ra.G = G;
     ra.mode = p->mode;
     ra.need_long = bif ? 1 : 0;
@@ -403,7 +422,7 @@ bf_status_t chunk_impl(const void* q, const void* k, const void* v, int32_t dtyp
     ra.Kl = Kl;
     std::memcpy(ra.omega, rope.omega, sizeof(ra.omega));
     std::memcpy(ra.omega_corr, rope.omega_corr, sizeof(ra.omega_corr));
-    bf::cache_rephase_kernel<128><<<static_cast<unsigned>((P0 + 7) / 8), 256, 0, st>>>(ra);
+    bf::cache_rephase_kernel<128><<<static_cast<unsigned>((P0 - j_begin + 7) / 8), 256, 0, st>>>(ra);
     if (cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
   }
   // 2. the chunk: RoPE forms of q and k at positions P0.., key rows P0.., cache rows P0..
@@ -449,13 +468,15 @@ bf_status_t chunk_impl(const void* q, const void* k, const void* v, int32_t dtyp
   ta.hq = p->hq;
   ta.hkv = p->hkv;
   ta.batch = 1;
-  ta.w0 = bif ? p->w0 : L;
+  ta.w0 = kind != bf::tc2::KIND_PLAIN ? p->w0 : L;
   ta.q_off = P0;
   ta.Lq = C;
   ta.scale_log2 = scale_log2(p);
   constexpr int smem = bf::attn_tc2_smem_bytes();
   const long long n_cta = static_cast<long long>((C + bf::tc::BM - 1) / bf::tc::BM) * (p->hq / 2);
-  auto kern = bif ? bf::attn_tc2_kernel<true> : bf::attn_tc2_kernel<false>;
+  auto kern = kind == bf::tc2::KIND_BIFOCAL  ? bf::attn_tc2_kernel<bf::tc2::KIND_BIFOCAL>
+              : kind == bf::tc2::KIND_WINDOW ? bf::attn_tc2_kernel<bf::tc2::KIND_WINDOW>
+                                        : bf::attn_tc2_kernel<bf::tc2::KIND_PLAIN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess) {
     kern<<<static_cast<unsigned>(n_cta), bf::tc2::NTHREADS2, smem, st>>>(ta);
@@ -502,12 +523,15 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
   if (p->hq / p->hkv > bf::dec::MAX_G) return BF_ERR_UNSUPPORTED;
   if (!aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16))
     return BF_ERR_INVALID;
+  const bool window = bifocal_api && (p->flags & BF_FLAG_WINDOW);
+  if (window && p->w0 < 1) return BF_ERR_INVALID;
   const DecodeLayout lay = decode_layout(L, p);
   if (!workspace || !aligned(workspace, 256) || ws_bytes < lay.total) return BF_ERR_WORKSPACE;
 
   const int D = p->head_dim;
   const int G = bifocal_api ? factor(L, p->w_pretrained) : 1;
-  const bool bif = bifocal_api && (G > 1 || (p->flags & BF_FLAG_FORCE_BIFOCAL)) && p->w0 < L;
+  const bool bif = !window && bifocal_api && (G > 1 || (p->flags & BF_FLAG_FORCE_BIFOCAL)) && p->w0 < L;
+  const int key0 = window ? std::max(0, L - p->w0) : 0;  // a window reads keys L - w0 .. L - 1 only
   const Rope rope = make_rope(p->rope_theta, D, G);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -536,9 +560,10 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
   const int head_groups = (p->hkv + bf::dec::HPC - 1) / bf::dec::HPC;
   const int sms = std::max(1, sm_count());
   const int target = std::max(1, std::min(kMaxSplits, sms / head_groups));
-  int split_len = (L + target - 1) / target;
+  const int n_keys = L - key0;
+  int split_len = (n_keys + target - 1) / target;
   split_len = (split_len + bf::dec::KB - 1) / bf::dec::KB * bf::dec::KB;
-  const int n_split = (L + split_len - 1) / split_len;
+  const int n_split = (n_keys + split_len - 1) / split_len;
   da.q = static_cast<const bf16*>(q);
   da.part_o = reinterpret_cast<float*>(ws + lay.part_o);
   da.part_ml = reinterpret_cast<float*>(ws + lay.part_ml);
@@ -549,6 +574,7 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
   da.G = G;
   da.mode = bifocal_api ? p->mode : 0;
   da.bifocal = bif ? 1 : 0;
+  da.key0 = key0;
   da.split_len = split_len;
   da.n_split = n_split;
   da.scale_log2 = scale_log2(p);

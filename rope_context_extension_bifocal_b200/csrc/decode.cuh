@@ -38,6 +38,7 @@ struct DecodeArgs {
   float* part_o;           // [2 * n_split, hq, D] unnormalised
   float* part_ml;          // [2 * n_split, hq, 2]: running max (log2 domain), sum
   int L, hq, hkv, w0, G, mode, bifocal;
+  int key0;  // first key read: 0, or L - w0 for a sliding window
   int split_len, n_split;
   float scale_log2;
   double omega[64];
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   const int nheads = min(HPC, a.hkv - head0);
   const int g = a.hq / a.hkv;
   const int p = a.L - 1;
-  const int jbeg = blockIdx.x * a.split_len;
+  const int jbeg = a.key0 + blockIdx.x * a.split_len;
   const int jend = min(a.L, jbeg + a.split_len);
   const int nstage = (jend - jbeg + KB - 1) / KB;
   const int local_from = a.bifocal ? max(0, a.L - a.w0) : 0;  // keys j >= local_from are local

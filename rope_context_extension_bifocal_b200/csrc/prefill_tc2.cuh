@@ -60,12 +60,16 @@ __device__ __forceinline__ int floordiv(int a, int b) { return a >= 0 ? a / b : 
 
 // Visit schedule of one query tile: n_lf fully long tiles (0..n_lf-1), then n_b band-edge
 // tiles, then the rest fully local. Visits: long tiles, long half of band tiles, [Q reload],
-// local half of band tiles (when w0 > 0), local tiles.
+// local half of band tiles (when w0 > 0), local tiles. The sliding-window kind drops the
+// long-range pairs: its visits start after the `skip` long ones.
+constexpr int KIND_PLAIN = 0, KIND_BIFOCAL = 1, KIND_WINDOW = 2;
+
 struct Schedule {
-  int n_kt, n_lf, n_b, n_bl, n_of;
-  __device__ __forceinline__ int n_long() const { return n_lf + n_b; }
-  __device__ __forceinline__ int total() const { return n_lf + n_b + n_bl + n_of; }
-  __device__ __forceinline__ void visit(int v, int& t, int& kind) const {
+  int n_kt, n_lf, n_b, n_bl, n_of, skip;
+  __device__ __forceinline__ int n_long() const { return n_lf + n_b - skip; }
+  __device__ __forceinline__ int total() const { return n_lf + n_b + n_bl + n_of - skip; }
+  __device__ __forceinline__ void visit(int vis, int& t, int& kind) const {
+    const int v = vis + skip;
     if (v < n_lf) {
       t = v;
       kind = LONG_FULL;
@@ -82,11 +86,12 @@ struct Schedule {
   }
 };
 
-template <bool BIFOCAL>
+template <int KIND>
 __device__ __forceinline__ Schedule make_schedule(int i0, int n_kt, int w0) {
   Schedule s;
   s.n_kt = n_kt;
-  if (!BIFOCAL) {
+  s.skip = 0;
+  if (KIND == KIND_PLAIN) {
     s.n_lf = s.n_b = s.n_bl = 0;
     s.n_of = n_kt;
     return s;
@@ -97,6 +102,7 @@ __device__ __forceinline__ Schedule make_schedule(int i0, int n_kt, int w0) {
   s.n_b = max(min(C, n_kt) - s.n_lf, 0);
   s.n_bl = w0 > 0 ? s.n_b : 0;
   s.n_of = n_kt - s.n_lf - s.n_b;
+  if (KIND == KIND_WINDOW) s.skip = s.n_lf + s.n_b;
   return s;
 }
 
@@ -117,7 +123,7 @@ struct Tc2Args {
   float scale_log2;
 };
 
-template <bool BIFOCAL>
+template <int KIND>
 __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __grid_constant__ Tc2Args a) {
   using namespace tc2;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -136,7 +142,7 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
   const int kvh = h0 / (a.hq / a.hkv);
   const int i0 = a.q_off + qt * BM;  // absolute position of the tile's first query row
   const int n_kt = (min(i0 + BM, a.q_off + a.Lq) + BN - 1) / BN;
-  const Schedule sch = make_schedule<BIFOCAL>(i0, n_kt, a.w0);
+  const Schedule sch = make_schedule<KIND>(i0, n_kt, a.w0);
   const int nv = sch.total();
   const bool has_long = sch.n_long() > 0;
   const bool has_orig = sch.n_bl + sch.n_of > 0;
@@ -184,7 +190,7 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
         prefetch_tensormap(&a.qo_map);
         prefetch_tensormap(&a.ko_map);
         prefetch_tensormap(&a.v_map);
-        if (BIFOCAL) {
+        if (KIND == KIND_BIFOCAL) {
           prefetch_tensormap(&a.ql_map);
           prefetch_tensormap(&a.kl_map);
         }
@@ -358,7 +364,12 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
       // reference m_ref. m_ref never exceeds the running max, so every P term is bounded by
       // 2^(running max - m_ref); the row sum bounds them all, and a sum above 2^24 (or not
       // finite) sends the visit to the exact two-pass path below.
-      bool exact = masked || m_ref == -INFINITY;
+      // Both choices below are made for the whole warp: each path reads S with tcgen05.ld,
+      // a warp-collective (.sync.aligned) instruction, so the lanes must not split between
+      // them. A row that needs the exact path (its reference is still -inf: no key of the
+      // earlier visits was in range, as happens in a sliding window; or its fast sum
+      // overflowed) takes the whole warp with it; the exact path is correct for every row.
+      bool exact = __any_sync(0xffffffffu, masked || m_ref == -INFINITY);
       if (!exact) {
         // pairs of columns go through the packed f32x2 FMA and add
         const uint64_t sc2 = f2_pack(sc, sc), nref2 = f2_pack(-m_ref, -m_ref);
@@ -383,7 +394,7 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
 #pragma unroll
         for (int u = 0; u < 4; ++u) f2_unpack(r4[u], r8[2 * u], r8[2 * u + 1]);
         rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
-        exact = !(rs <= 16777216.f);
+        exact = __any_sync(0xffffffffu, !(rs <= 16777216.f));
       }
       if (exact) {
         // pass 1: raw row max over the 128 columns

@@ -192,6 +192,7 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
 struct RephaseArgs {
   const __nv_bfloat16* kcache;  // [Lc, hkv, D], rows 0 .. P0-1 read
   int P0, hkv, Lk;              // cached rows; kv heads; rows of Ko / Kl per kv head
+  int j_begin;                  // first cached row needed (0, or the window's first tile)
   int G, mode, need_long;
   __half* Ko;                   // [hkv, Lk, D]
   __half* Kl;
@@ -206,7 +207,7 @@ __global__ void __launch_bounds__(256) cache_rephase_kernel(const __grid_constan
   constexpr int NPAIR = 8;
   constexpr int LANES_PER_ROW = P / NPAIR;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long j_ll = static_cast<long long>(blockIdx.x) * 8 + warp;
+  const long long j_ll = a.j_begin + static_cast<long long>(blockIdx.x) * 8 + warp;
   if (j_ll >= a.P0) return;
   const int j = static_cast<int>(j_ll);
   const int grp = lane >> 3, l8 = lane & 7;

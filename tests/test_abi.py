@@ -157,6 +157,23 @@ def test_chunk_validation_before_launch(lib):
     assert call(params(), wsb=256) == 5
 
 
+def test_window_flag_validation_before_launch(lib):
+    W = bfl.FLAG_WINDOW
+
+    def prefill(p):
+        return lib.bifocal_prefill(FAKE, FAKE, FAKE, 0, 1, 128, ctypes.byref(p), FAKE, None, None, None, FAKE, 0, None)
+
+    def decode(p):
+        return lib.bifocal_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 200, 100, ctypes.byref(p), FAKE, None, FAKE, 0, None)
+
+    assert prefill(params(w0=0, flags=W)) == 1             # an empty window
+    assert prefill(params(w0=64, head_dim=64, flags=W)) == 2  # the window runs on the D = 128 ping-pong kernel
+    assert prefill(params(w0=64, hq=24, flags=W)) == 2      # odd GQA group
+    assert prefill(params(w0=64, flags=W)) == 5             # valid: stops at the (empty) workspace
+    assert decode(params(w0=0, flags=W)) == 1
+    assert decode(params(w0=64, flags=W)) == 5
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     mod = importlib.import_module("rope_context_extension_bifocal_b200")
