@@ -132,6 +132,20 @@ BF_API bf_status_t bifocal_prefill_attention(const void* v, int32_t dtype, int32
                                              const bf_params_t* p, void* out, float* lse, void* workspace,
                                              size_t ws_bytes, void* stream);
 
+/* Step 1 with the step before the path fused in: the per-head RMS norm of the model's attention
+ * block (Qwen3's q_norm and k_norm) applied to q and k inside the RoPE pass, so the normalised
+ * q and k are never written. Row x of every query head (key head) becomes
+ * x * rsqrt(mean_d(x_d^2) + eps) * q_norm_w (k_norm_w), in fp32, before the rotations; kcache_out
+ * then holds the normalised keys under the original RoPE. The pages say nothing about norms:
+ * this serves the Qwen3 models they evaluate.
+ *   q_norm_w, k_norm_w [D] in the input dtype, device pointers (16-byte aligned for bf16, 32 for fp32);
+ *   eps >= 0. Follow with bifocal_prefill_attention. Other arguments and errors as bifocal_prefill_rope;
+ *   BF_ERR_INVALID also for NULL weights or a negative or non-finite eps. */
+BF_API bf_status_t bifocal_prefill_rope_qknorm(const void* q, const void* k, const void* v, int32_t dtype,
+                                               int32_t batch, int32_t L, const bf_params_t* p, const void* q_norm_w,
+                                               const void* k_norm_w, float eps, void* kcache_out, void* vcache_out,
+                                               void* workspace, size_t ws_bytes, void* stream);
+
 /* Plain causal attention under the original RoPE: the same kernels with the long branch
  * compiled out (the comparator for the bifocal overhead). Same arguments as bifocal_prefill;
  * w0, w_pretrained and mode are ignored. */

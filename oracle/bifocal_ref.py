@@ -437,3 +437,13 @@ def sliding_window_cached_reference(q, kcache, vcache, P0: int, window: int, the
             out[n, h] = (e @ vc[:, kvh]) / e.sum()
             lse[h, n] = m + math.log(e.sum())
     return out, lse
+
+
+# ----------------------------------------------------------------------------------
+# Per-head RMS norm of q and k (Qwen3's q_norm / k_norm, the step before the path)
+# ----------------------------------------------------------------------------------
+def qk_rms_norm(x, weight, eps: float):
+    """x [..., D] -> x / sqrt(mean_d x^2 + eps) * weight, fp64, over the last axis."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(weight, dtype=np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * w

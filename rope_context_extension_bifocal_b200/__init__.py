@@ -71,6 +71,9 @@ def _lib() -> ctypes.CDLL:
             getattr(L, name).argtypes, getattr(L, name).restype = pre, i32
         L.bifocal_prefill_rope.argtypes = [vp, vp, vp, i32, i32, i32, pp, vp, vp, vp, sz, vp]
         L.bifocal_prefill_rope.restype = i32
+        L.bifocal_prefill_rope_qknorm.argtypes = [vp, vp, vp, i32, i32, i32, pp, vp, vp, ctypes.c_float, vp, vp,
+                                                  vp, sz, vp]
+        L.bifocal_prefill_rope_qknorm.restype = i32
         L.bifocal_prefill_attention.argtypes = [vp, i32, i32, i32, pp, vp, vp, vp, sz, vp]
         L.bifocal_prefill_attention.restype = i32
         L.bifocal_prefill_chunk_workspace_size.argtypes = [i32, i32, pp]
@@ -189,6 +192,16 @@ def bifocal_prefill_rope(q, k, v, params: Params, workspace, kcache=None, vcache
                                      ctypes.byref(params), _ptr(kcache), _ptr(vcache), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "bifocal_prefill_rope")
+
+
+def bifocal_prefill_rope_qknorm(q, k, v, params: Params, workspace, q_norm_w, k_norm_w, eps: float = 1e-6,
+                                kcache=None, vcache=None, stream=None):
+    """Step 1 with Qwen3's per-head q/k RMS norm fused in (weights [D], input dtype)."""
+    st = _lib().bifocal_prefill_rope_qknorm(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), q.shape[0], q.shape[1],
+                                            ctypes.byref(params), _ptr(q_norm_w), _ptr(k_norm_w), float(eps),
+                                            _ptr(kcache), _ptr(vcache), _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "bifocal_prefill_rope_qknorm")
 
 
 def bifocal_prefill_attention(v, params: Params, workspace, out, lse=None, batch=None, L=None, dtype=None,

@@ -209,7 +209,8 @@ bf_status_t plan_prefill(bool bifocal_api, int32_t dtype, int32_t batch, int32_t
 
 bf_status_t prefill_rope_impl(bool bifocal_api, const void* q, const void* k, const void* v, int32_t dtype,
                               int32_t batch, int32_t L, const bf_params_t* p, void* kcache_out, void* vcache_out,
-                              void* workspace, size_t ws_bytes, void* stream) {
+                              void* workspace, size_t ws_bytes, void* stream, const void* q_norm_w = nullptr,
+                              const void* k_norm_w = nullptr, float norm_eps = 0.f) {
   PrefillPlan plan;
   bf_status_t s = check_params(p, bifocal_api);
   if (s != BF_OK) return s;
@@ -246,6 +247,9 @@ bf_status_t prefill_rope_impl(bool bifocal_api, const void* q, const void* k, co
   pa.vcache = static_cast<bf16*>(vcache_out);
   std::memcpy(pa.omega, plan.rope.omega, sizeof(pa.omega));
   std::memcpy(pa.omega_long, plan.rope.omega_long, sizeof(pa.omega_long));
+  pa.q_norm_w = q_norm_w;
+  pa.k_norm_w = k_norm_w;
+  pa.norm_eps = norm_eps;
   const long long rows = static_cast<long long>(batch) * L;
   const dim3 pgrid(static_cast<unsigned>((rows + 7) / 8));
   if (dtype == BF_DTYPE_BF16) {
@@ -671,6 +675,17 @@ bf_status_t bifocal_prefill_rope(const void* q, const void* k, const void* v, in
                                  int32_t L, const bf_params_t* p, void* kcache_out, void* vcache_out, void* workspace,
                                  size_t ws_bytes, void* stream) {
   return prefill_rope_impl(true, q, k, v, dtype, batch, L, p, kcache_out, vcache_out, workspace, ws_bytes, stream);
+}
+
+bf_status_t bifocal_prefill_rope_qknorm(const void* q, const void* k, const void* v, int32_t dtype, int32_t batch,
+                                        int32_t L, const bf_params_t* p, const void* q_norm_w, const void* k_norm_w,
+                                        float eps, void* kcache_out, void* vcache_out, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  if (!q_norm_w || !k_norm_w || !(eps >= 0.f) || !std::isfinite(eps)) return BF_ERR_INVALID;
+  const size_t align_in = dtype == BF_DTYPE_FP32 ? 32 : 16;
+  if (!aligned(q_norm_w, align_in) || !aligned(k_norm_w, align_in)) return BF_ERR_INVALID;
+  return prefill_rope_impl(true, q, k, v, dtype, batch, L, p, kcache_out, vcache_out, workspace, ws_bytes, stream,
+                           q_norm_w, k_norm_w, eps);
 }
 
 bf_status_t bifocal_prefill_attention(const void* v, int32_t dtype, int32_t batch, int32_t L, const bf_params_t* p,

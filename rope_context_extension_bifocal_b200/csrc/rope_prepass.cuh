@@ -14,6 +14,9 @@
 // caller's kcache in [b, Lc, hkv, D] when asked. fp32 inputs are rounded to bf16 here.
 // A chunk over an existing cache passes its first absolute position in pos0: the angles,
 // the key rows and the cache rows are those of positions pos0 .. pos0 + L - 1.
+// With q_norm_w / k_norm_w the pass first applies the per-head RMS norm of the model's
+// attention block (Qwen3 normalises every query and key head over D with a learned weight
+// before RoPE), so the step before the path costs no extra pass over q and k.
 //
 // cache_rephase_kernel prepares the cached part of a chunked prefill: the cache holds
 // keys under the original RoPE (bf16), so Ko is their fp16 copy (exact: a bf16 value
@@ -46,6 +49,11 @@ struct PrepassArgs {
   __nv_bfloat16* vcache;   // optional [b, L, hkv, D]
   double omega[64];        // omega_k = theta^(-2k/D)
   double omega_long[64];   // omega_k / G (frequency interpolation)
+  // optional per-head RMS norm before the rotation (Qwen3's q_norm / k_norm): x <- x *
+  // rsqrt(mean_d(x^2) + eps) * w[d], weights [D] in the input dtype; null = no norm
+  const void* q_norm_w;
+  const void* k_norm_w;
+  float norm_eps;
 };
 
 template <typename T>
@@ -137,10 +145,36 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
     Vec8<Tin> x1, x2;
     x1.load(src + k0);
     x2.load(src + P + k0);
+    float xu[8], xw[8];
+#pragma unroll
+    for (int i = 0; i < NPAIR; ++i) {
+      xu[i] = x1.get(i);
+      xw[i] = x2.get(i);
+    }
+    const void* nw = is_q ? a.q_norm_w : a.k_norm_w;
+    if (nw) {
+      // RMS over the row's D elements: this lane holds 16 (D = 128) or 8 of the row's pairs'
+      // elements; the row's lanes are the LANES_PER_ROW lanes of this group
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < NPAIR; ++i) ss += xu[i] * xu[i] + xw[i] * xw[i];
+      const unsigned gmask = ((1u << LANES_PER_ROW) - 1u) << (grp * 8);
+#pragma unroll
+      for (int off = LANES_PER_ROW / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(gmask, ss, off);
+      const float inv = rsqrtf(ss / D + a.norm_eps);
+      Vec8<Tin> w1, w2;
+      w1.load(static_cast<const Tin*>(nw) + k0);
+      w2.load(static_cast<const Tin*>(nw) + P + k0);
+#pragma unroll
+      for (int i = 0; i < NPAIR; ++i) {
+        xu[i] *= inv * w1.get(i);
+        xw[i] *= inv * w2.get(i);
+      }
+    }
     float yo1[8], yo2[8], yl1[8], yl2[8];
 #pragma unroll
     for (int i = 0; i < NPAIR; ++i) {
-      const float u = x1.get(i), w = x2.get(i);
+      const float u = xu[i], w = xw[i];
       yo1[i] = u * co[i] - w * so[i];
       yo2[i] = w * co[i] + u * so[i];
       yl1[i] = u * cl[i] - w * sl[i];

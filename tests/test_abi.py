@@ -174,6 +174,20 @@ def test_window_flag_validation_before_launch(lib):
     assert decode(params(w0=64, flags=W)) == 5
 
 
+def test_qknorm_validation_before_launch(lib):
+    f = lib.bifocal_prefill_rope_qknorm
+
+    def call(p, qw=FAKE, kw=FAKE, eps=1e-6, ws=FAKE, wsb=0):
+        return f(FAKE, FAKE, FAKE, 0, 1, 128, ctypes.byref(p), qw, kw, ctypes.c_float(eps), None, None, ws, wsb, None)
+
+    assert call(params(), qw=None) == 1
+    assert call(params(), kw=None) == 1
+    assert call(params(), eps=-1.0) == 1
+    assert call(params(), eps=float("nan")) == 1
+    assert call(params(), qw=FAKE + 2) == 1  # misaligned weights
+    assert call(params()) == 5               # valid: stops at the (empty) workspace
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     mod = importlib.import_module("rope_context_extension_bifocal_b200")
