@@ -414,6 +414,11 @@ def run_ours(args):
         torch.cuda.empty_cache()
         decode = run_decode(args, torch, bfl, si, dev, peaks, peak_kind)
 
+    paged = None
+    if not args.no_paged:
+        torch.cuda.empty_cache()
+        paged = run_paged(args, torch, bfl, si, dev, peaks, peak_kind)
+
     # ---- CPU baseline: the oracle on a bounded sample, rank 0, N = 1 only
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
@@ -442,6 +447,7 @@ def run_ours(args):
         "decode": decode,
         "chunked_prefill": chunk,
         "window_prefill": window,
+        "paged_decode": paged,
         "build": bfl.build_info(),
     }
     if dist.rank == 0:
@@ -518,6 +524,47 @@ def run_decode(args, torch, bfl, si, dev, peaks, peak_kind):
     }
 
 
+def run_paged(args, torch, bfl, si, dev, peaks, peak_kind):
+    """Batched decode over a paged cache: 8 sequences of ~16K tokens (Qwen3-8B heads), page 64."""
+    B, page, hq, hkv, D, w0, wp = 8, 64, 32, 8, 128, 4096, 4096
+    lens = [16384 + 97 * b for b in range(B)]  # G = 4 or 5 per sequence
+    max_len = max(lens) + 1
+    max_pages = (max_len + page - 1) // page
+    g = si.generator(404)
+    pool_pages = B * max_pages
+    table = torch.randperm(pool_pages, generator=g).to(torch.int32).reshape(B, max_pages).to(dev)
+    kpool = torch.randn(pool_pages * page, hkv, D, device=dev).to(torch.bfloat16)
+    vpool = torch.randn(pool_pages * page, hkv, D, device=dev).to(torch.bfloat16)
+    seq = torch.tensor(lens, dtype=torch.int32, device=dev)
+    q = torch.randn(B, hq, D, device=dev).to(torch.bfloat16)
+    kn = torch.randn(B, hkv, D, device=dev).to(torch.bfloat16)
+    vn = torch.randn(B, hkv, D, device=dev).to(torch.bfloat16)
+    prm = bfl.make_params(hq, hkv, D, w0, wp, 1e6)
+    ws = torch.empty(bfl.decode_paged_workspace_size(B, max_len, prm), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, hq, D, dtype=torch.bfloat16, device=dev)
+
+    def step():
+        bfl.bifocal_decode_paged(q, kn, vn, kpool, vpool, page, table, seq, max_len, w0=w0, w_pretrained=wp,
+                                 theta=1e6, want_lse=False, out=out, workspace=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(30)]
+    for a, b_ in ev:
+        a.record()
+        step()
+        b_.record()
+    torch.cuda.synchronize()
+    us = statistics.median(a.elapsed_time(b_) * 1e3 for a, b_ in ev)
+    nbytes = sum(4 * hkv * D * L for L in lens)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    return {"workload": f"qwen3_8b_paged_decode_B{B}_L{lens[0]}-{lens[-1]}_page{page}", "us_median": us,
+            "gbs": gbs, "frac_of_hbm": gbs / hbm, "bytes_per_step": nbytes,
+            "G": [bfl.bifocal_factor(L, wp) for L in lens]}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -529,6 +576,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-chunk", action="store_true")
     ap.add_argument("--no-window", action="store_true")
+    ap.add_argument("--no-paged", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -200,6 +200,33 @@ BF_API bf_status_t bifocal_decode(const void* q, const void* k_new, const void* 
                            int32_t cap, int32_t L, const bf_params_t* p, void* out, float* lse, void* workspace,
                            size_t ws_bytes, void* stream);
 
+/* One decode step for a batch of sequences over a paged cache (vLLM-style block tables), each
+ * sequence at its own length, with its own G = max(1, ceil(L_b / w_pretrained)), band edge and
+ * correction rotation ([AF] module 2: the factor follows each sequence's current length).
+ *   q      [batch, hq, D] bf16 raw queries of the new tokens; k_new, v_new [batch, hkv, D] bf16 raw
+ *   kpool, vpool [pool_pages * page_size, hkv, D] bf16: the pages; keys under the ORIGINAL RoPE
+ *   block_table [batch, max_pages] int32 (device): sequence b's logical key j is pool row
+ *          block_table[b * max_pages + j / page_size] * page_size + j % page_size
+ *   seq_lens [batch] int32 (device): L_b, the length with the new token, 1 <= L_b <= max_len;
+ *          the new token's key and value are written at logical position L_b - 1
+ *   max_len: an upper bound of every L_b (host); it sets the split layout and the workspace
+ *   page_size: a multiple of 16 (one 16-key stage never straddles two pages)
+ *   out [batch, hq, D] bf16;  lse [batch, hq] fp32 (may be NULL)
+ *   workspace / ws_bytes: >= bifocal_decode_paged_workspace_size(batch, max_len, p), 256-byte aligned.
+ * Pages past a sequence's length are never read except the tail of its last 16-key stage, whose
+ * keys are masked and whose values are zeroed in shared memory before use (an uninitialised
+ * slot cannot turn the result into NaN). block_table entries and seq_lens are trusted: each
+ * used entry must name a page of the pool.
+ * Errors: as bifocal_decode; BF_ERR_INVALID also for batch, pool_pages, max_pages or max_len < 1, a
+ * page_size that is not a positive multiple of 16, max_pages * page_size < max_len or a NULL
+ * table; BF_ERR_UNSUPPORTED for BF_FLAG_WINDOW. */
+BF_API size_t bifocal_decode_paged_workspace_size(int32_t batch, int32_t max_len, const bf_params_t* p);
+BF_API bf_status_t bifocal_decode_paged(const void* q, const void* k_new, const void* v_new, void* kpool,
+                                        void* vpool, int32_t pool_pages, int32_t page_size,
+                                        const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
+                                        int32_t max_len, int32_t batch, const bf_params_t* p, void* out,
+                                        float* lse, void* workspace, size_t ws_bytes, void* stream);
+
 /* bifocal_decode without a caller workspace, for callers that cannot allocate device memory
  * themselves: for example a plug-in hosted by a runtime that owns and pre-plans all device
  * memory, or a latency-critical loop that may not call cudaMalloc (which synchronises the

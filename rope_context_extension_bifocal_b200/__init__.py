@@ -83,6 +83,11 @@ def _lib() -> ctypes.CDLL:
         dec = [vp, vp, vp, vp, vp, i32, i32, pp, vp, vp, vp, sz, vp]
         for name in ("bifocal_decode", "rope_causal_decode"):
             getattr(L, name).argtypes, getattr(L, name).restype = dec, i32
+        L.bifocal_decode_paged_workspace_size.argtypes = [i32, i32, pp]
+        L.bifocal_decode_paged_workspace_size.restype = sz
+        L.bifocal_decode_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, i32, vp, i32, i32, pp, vp, vp, vp, sz,
+                                           vp]
+        L.bifocal_decode_paged.restype = i32
         L.bifocal_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, pp, vp, vp, vp]
         L.bifocal_decode_noalloc.restype = i32
         L.bifocal_status_string.argtypes, L.bifocal_status_string.restype = [i32], ctypes.c_char_p
@@ -289,6 +294,32 @@ def bifocal_decode_noalloc(q, k_new, v_new, kcache, vcache, L: int, *, w0: int, 
                                        _ptr(lse if want_lse else None), _stream(stream))
     _check(st, "bifocal_decode_noalloc")
     return out, (lse if want_lse else None)
+
+
+def decode_paged_workspace_size(batch: int, max_len: int, params: Params) -> int:
+    return int(_lib().bifocal_decode_paged_workspace_size(int(batch), int(max_len), ctypes.byref(params)))
+
+
+def bifocal_decode_paged(q, k_new, v_new, kpool, vpool, page_size: int, block_table, seq_lens, max_len: int, *,
+                         w0: int, w_pretrained: int, theta: float, mode: str = FREQ_INTERP,
+                         scale: Optional[float] = None, flags: int = 0, want_lse: bool = True, out=None,
+                         workspace=None, stream=None):
+    """Batched decode over a paged cache. q [B, Hq, D], k_new / v_new [B, Hkv, D] bf16; kpool / vpool
+    [pages * page_size, Hkv, D] bf16; block_table [B, max_pages] int32 and seq_lens [B] int32 on the
+    device (lengths with the new token); max_len bounds them. Returns (out [B, Hq, D], lse [B, Hq])."""
+    import torch
+    B, hq, D = q.shape
+    p = make_params(hq, k_new.shape[1], D, w0, w_pretrained, theta, mode, scale, flags)
+    out = torch.empty(B, hq, D, dtype=torch.bfloat16, device=q.device) if out is None else out
+    lse = torch.empty(B, hq, dtype=torch.float32, device=q.device) if want_lse else None
+    ws = _workspace(decode_paged_workspace_size(B, max_len, p), q.device) if workspace is None else workspace
+    pool_pages = kpool.shape[0] // page_size
+    st = _lib().bifocal_decode_paged(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(kpool), _ptr(vpool), pool_pages,
+                                     int(page_size), _ptr(block_table), block_table.shape[1], _ptr(seq_lens),
+                                     int(max_len), B, ctypes.byref(p), _ptr(out), _ptr(lse), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "bifocal_decode_paged")
+    return out, lse
 
 
 def rope_causal_decode(q, k_new, v_new, kcache, vcache, L: int, *, theta: float, scale: Optional[float] = None,

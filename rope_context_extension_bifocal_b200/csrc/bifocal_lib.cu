@@ -609,9 +609,11 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
   bf16* o16 = static_cast<bf16*>(out);
   const dim3 cblock(32 * bf::COMBINE_WARPS);
   if (D == 128)
-    e = launch_pdl(bf::decode_combine_kernel<128>, dim3(p->hq, 128 / 32), cblock, 0, st, po, pml, nparts, hq, o16, lse);
+    e = launch_pdl(bf::decode_combine_kernel<128>, dim3(p->hq, 128 / 32), cblock, 0, st, po, pml, nparts, hq, o16, lse,
+                   static_cast<const int*>(nullptr), 0, 0);
   else
-    e = launch_pdl(bf::decode_combine_kernel<64>, dim3(p->hq, 64 / 32), cblock, 0, st, po, pml, nparts, hq, o16, lse);
+    e = launch_pdl(bf::decode_combine_kernel<64>, dim3(p->hq, 64 / 32), cblock, 0, st, po, pml, nparts, hq, o16, lse,
+                   static_cast<const int*>(nullptr), 0, 0);
   return e == cudaSuccess ? BF_OK : BF_ERR_CUDA;
 }
 
@@ -640,6 +642,123 @@ void* noalloc_scratch_ptr() {
 
 }  // namespace
 
+// ------------------------------------------------------------------ batched decode over a paged cache
+// Partial rows per sequence: two per split, splits <= min(kMaxSplits, ceil(max_len / KB)).
+int paged_parts_stride(int max_len) { return 2 * std::min(kMaxSplits, (max_len + bf::dec::KB - 1) / bf::dec::KB); }
+
+size_t paged_workspace(int batch, int max_len, const bf_params_t* p) {
+  const size_t rows = static_cast<size_t>(batch) * paged_parts_stride(max_len) * p->hq;
+  return align256(rows * p->head_dim * 4) + align256(rows * 2 * 4);
+}
+
+bf_status_t decode_paged_impl(const void* q, const void* k_new, const void* v_new, void* kpool, void* vpool,
+                              int32_t pool_pages, int32_t page_size, const int32_t* block_table, int32_t max_pages,
+                              const int32_t* seq_lens, int32_t max_len, int32_t batch, const bf_params_t* p,
+                              void* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  bf_status_t s = check_params(p, true);
+  if (s != BF_OK) return s;
+  if (!q || !k_new || !v_new || !kpool || !vpool || !block_table || !seq_lens || !out) return BF_ERR_INVALID;
+  if (batch < 1 || pool_pages < 1 || max_pages < 1 || max_len < 1) return BF_ERR_INVALID;
+  if (page_size < bf::dec::KB || page_size % bf::dec::KB) return BF_ERR_INVALID;
+  if (static_cast<int64_t>(max_pages) * page_size < max_len ||
+      static_cast<int64_t>(pool_pages) * page_size > 0x7fffffffLL)
+    return BF_ERR_INVALID;
+  if (p->hq / p->hkv > bf::dec::MAX_G) return BF_ERR_UNSUPPORTED;
+  if (p->flags & BF_FLAG_WINDOW) return BF_ERR_UNSUPPORTED;
+  if (!aligned(kpool, 16) || !aligned(vpool, 16) || !aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) ||
+      !aligned(block_table, 4) || !aligned(seq_lens, 4) || !aligned(out, 16) || (lse && !aligned(lse, 4)))
+    return BF_ERR_INVALID;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < paged_workspace(batch, max_len, p)) return BF_ERR_WORKSPACE;
+
+  const int D = p->head_dim;
+  const Rope rope = make_rope(p->rope_theta, D, 1);  // omega only: G is each sequence's own
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int stride = paged_parts_stride(max_len);
+  const size_t rows = static_cast<size_t>(batch) * stride * p->hq;
+  float* part_o = reinterpret_cast<float*>(ws);
+  float* part_ml = reinterpret_cast<float*>(ws + align256(rows * D * 4));
+
+  // 1. append every sequence's new token at its own position
+  bf::AppendArgs ap{};
+  ap.k_new = static_cast<const bf16*>(k_new);
+  ap.v_new = static_cast<const bf16*>(v_new);
+  ap.kcache = static_cast<bf16*>(kpool);
+  ap.vcache = static_cast<bf16*>(vpool);
+  ap.hkv = p->hkv;
+  ap.seq_lens = seq_lens;
+  ap.block_table = block_table;
+  ap.max_pages = max_pages;
+  ap.page_size = page_size;
+  std::memcpy(ap.omega, rope.omega, sizeof(ap.omega));
+  if (D == 128)
+    bf::decode_append_kernel<128><<<dim3(p->hkv, batch), 32, 0, st>>>(ap);
+  else
+    bf::decode_append_kernel<64><<<dim3(p->hkv, batch), 32, 0, st>>>(ap);
+  if (cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
+
+  // 2. split-KV partials: one split length for the batch (from max_len), a grid of about one
+  //    CTA per SM in total; CTAs past a shorter sequence's end leave at once
+  bf::DecodeArgs da;
+  std::memset(&da, 0, sizeof(da));
+  const int cap = pool_pages * page_size;
+  if (!make_cache_map(&da.kmap, kpool, cap, p->hkv, D, bf::dec::KB) ||
+      !make_cache_map(&da.vmap, vpool, cap, p->hkv, D, bf::dec::KB))
+    return BF_ERR_CUDA;
+  const int head_groups = (p->hkv + bf::dec::HPC - 1) / bf::dec::HPC;
+  const int sms = std::max(1, sm_count());
+  const int target = std::max(1, std::min(kMaxSplits, sms / (head_groups * batch)));
+  int split_len = (max_len + target - 1) / target;
+  split_len = (split_len + bf::dec::KB - 1) / bf::dec::KB * bf::dec::KB;
+  const int n_split = (max_len + split_len - 1) / split_len;
+  da.q = static_cast<const bf16*>(q);
+  da.part_o = part_o;
+  da.part_ml = part_ml;
+  da.L = max_len;
+  da.hq = p->hq;
+  da.hkv = p->hkv;
+  da.w0 = p->w0;
+  da.mode = p->mode;
+  da.split_len = split_len;
+  da.n_split = n_split;
+  da.scale_log2 = scale_log2(p);
+  std::memcpy(da.omega, rope.omega, sizeof(da.omega));
+  da.seq_lens = seq_lens;
+  da.block_table = block_table;
+  da.max_pages = max_pages;
+  da.page_size = page_size;
+  da.w_pretrained = p->w_pretrained;
+  da.force_bifocal = (p->flags & BF_FLAG_FORCE_BIFOCAL) ? 1 : 0;
+  da.parts_stride = stride;
+  const dim3 grid(n_split, head_groups, batch);
+  cudaError_t e;
+  if (D == 128) {
+    constexpr int smem = bf::decode_smem_bytes<128>();
+    e = cudaFuncSetAttribute(bf::decode_partial_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+      e = launch_pdl(bf::decode_partial_kernel<128>, grid, dim3(bf::decode_threads<128>()), smem, st, da);
+  } else {
+    constexpr int smem = bf::decode_smem_bytes<64>();
+    e = cudaFuncSetAttribute(bf::decode_partial_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+      e = launch_pdl(bf::decode_partial_kernel<64>, grid, dim3(bf::decode_threads<64>()), smem, st, da);
+  }
+  if (e != cudaSuccess) return BF_ERR_CUDA;
+
+  // 3. combine per sequence
+  const dim3 cblock(32 * bf::COMBINE_WARPS);
+  bf16* o16 = static_cast<bf16*>(out);
+  if (D == 128)
+    e = launch_pdl(bf::decode_combine_kernel<128>, dim3(p->hq, 128 / 32, batch), cblock, 0, st,
+                   static_cast<const float*>(part_o), static_cast<const float*>(part_ml), 2 * n_split, p->hq, o16,
+                   lse, static_cast<const int*>(seq_lens), split_len, stride);
+  else
+    e = launch_pdl(bf::decode_combine_kernel<64>, dim3(p->hq, 64 / 32, batch), cblock, 0, st,
+                   static_cast<const float*>(part_o), static_cast<const float*>(part_ml), 2 * n_split, p->hq, o16,
+                   lse, static_cast<const int*>(seq_lens), split_len, stride);
+  return e == cudaSuccess ? BF_OK : BF_ERR_CUDA;
+}
+
 extern "C" {
 
 int32_t bifocal_factor(int64_t L, int32_t w_pretrained) {
@@ -658,6 +777,19 @@ bf_status_t bifocal_prefill(const void* q, const void* k, const void* v, int32_t
                             void* workspace, size_t ws_bytes, void* stream) {
   return prefill_impl(true, q, k, v, dtype, batch, L, p, out, lse, kcache_out, vcache_out, workspace, ws_bytes,
                       stream);
+}
+
+size_t bifocal_decode_paged_workspace_size(int32_t batch, int32_t max_len, const bf_params_t* p) {
+  if (check_params(p, true) != BF_OK || batch < 1 || max_len < 1) return 0;
+  return paged_workspace(batch, max_len, p);
+}
+
+bf_status_t bifocal_decode_paged(const void* q, const void* k_new, const void* v_new, void* kpool, void* vpool,
+                                 int32_t pool_pages, int32_t page_size, const int32_t* block_table, int32_t max_pages,
+                                 const int32_t* seq_lens, int32_t max_len, int32_t batch, const bf_params_t* p,
+                                 void* out, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  return decode_paged_impl(q, k_new, v_new, kpool, vpool, pool_pages, page_size, block_table, max_pages, seq_lens,
+                           max_len, batch, p, out, lse, workspace, ws_bytes, stream);
 }
 
 size_t bifocal_prefill_chunk_workspace_size(int32_t P0, int32_t C, const bf_params_t* p) {

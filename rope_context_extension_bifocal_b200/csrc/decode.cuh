@@ -44,6 +44,14 @@ struct DecodeArgs {
   double omega[64];
   double omega_long[64];  // omega / G
   double omega_corr[64];  // omega * (1/G - 1)
+  // Batched form over a paged cache (grid.z = sequence; null seq_lens = the single call above):
+  // sequence b has length seq_lens[b] (with its new token); its logical key j lives in pool
+  // row block_table[b * max_pages + j / page_size] * page_size + j % page_size. G, the band
+  // edge and the long-range tables follow each sequence's own length.
+  const int* seq_lens;
+  const int* block_table;
+  int max_pages, page_size, w_pretrained, force_bifocal;
+  int parts_stride;  // partial rows reserved per sequence
 };
 
 // 128-byte swizzle of TMA SWIZZLE_128B: 16-byte chunk c of row r sits at chunk c ^ (r & 7).
@@ -77,11 +85,20 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   const int head0 = blockIdx.y * HPC;
   const int nheads = min(HPC, a.hkv - head0);
   const int g = a.hq / a.hkv;
-  const int p = a.L - 1;
+  const bool paged = a.seq_lens != nullptr;
+  const int bz = paged ? static_cast<int>(blockIdx.z) : 0;
+  const int L = paged ? a.seq_lens[bz] : a.L;
+  const int G = paged ? (L <= a.w_pretrained ? 1 : (L + a.w_pretrained - 1) / a.w_pretrained) : a.G;
+  const bool bifocal = paged ? ((G > 1 || a.force_bifocal) && a.w0 < L) : (a.bifocal != 0);
+  const int p = L - 1;
   const int jbeg = a.key0 + blockIdx.x * a.split_len;
-  const int jend = min(a.L, jbeg + a.split_len);
+  if (jbeg >= L) return;  // a shorter sequence of the batch: no keys in this split (the combine skips it)
+  const int jend = min(L, jbeg + a.split_len);
   const int nstage = (jend - jbeg + KB - 1) / KB;
-  const int local_from = a.bifocal ? max(0, a.L - a.w0) : 0;  // keys j >= local_from are local
+  const int local_from = bifocal ? max(0, L - a.w0) : 0;  // keys j >= local_from are local
+  // long-range tables: the host's for a single call, the same fp64 expressions per sequence when batched
+  auto omega_long = [&](int k) { return paged ? a.omega[k] / G : a.omega_long[k]; };
+  auto omega_corr = [&](int k) { return paged ? a.omega[k] / G - a.omega[k] : a.omega_corr[k]; };
   const int nconsumers = 2 * nheads;  // two warps per kv head, one 8-key n-tile of each stage each
 
   if (threadIdx.x == 0) {
@@ -107,12 +124,16 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
         // Only row p (the new token) comes from the append kernel; every other row was in the
         // cache before this step, so only the stage holding p waits for that grid.
         if (j0 + KB > p) pdl_wait();
+        // pool row of logical key j0 (pages hold a multiple of KB keys, so a stage is one page's)
+        const int row = paged ? a.block_table[static_cast<long long>(bz) * a.max_pages + j0 / a.page_size] * a.page_size +
+                                    j0 % a.page_size
+                              : j0;
         mbar_arrive_expect_tx(&full[st], bytes);
         for (int hh = 0; hh < nheads; ++hh)
           for (int hf = 0; hf < HALVES; ++hf) {
             const uint32_t off = st * STAGE_KV + (hh * HALVES + hf) * HEAD_TILE;
-            tma_load_4d(sK + off, &a.kmap, &full[st], 0, hf, head0 + hh, j0);
-            tma_load_4d(sV + off, &a.vmap, &full[st], 0, hf, head0 + hh, j0);
+            tma_load_4d(sK + off, &a.kmap, &full[st], 0, hf, head0 + hh, row);
+            tma_load_4d(sV + off, &a.vmap, &full[st], 0, hf, head0 + hh, row);
           }
       }
     }
@@ -131,7 +152,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
       fi_c[e] = pa_c[e] = 1.f;
       fi_s[e] = pa_s[e] = 0.f;
       if (pr < P) {
-        angle_cos_sin(a.omega_corr[pr], fi_c[e], fi_s[e]);
+        angle_cos_sin(omega_corr(pr), fi_c[e], fi_s[e]);
         angle_cos_sin(-a.omega[pr], pa_c[e], pa_s[e]);
       }
     }
@@ -150,8 +171,8 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
 #pragma unroll
           for (int hk = 0; hk < 2; ++hk) {
             const int jc = j0 + 8 * hk;
-            const double ang0 = (a.mode == 0) ? static_cast<double>(jc) * a.omega_corr[pr]
-                                              : static_cast<double>(jc / a.G - jc) * a.omega[pr];
+            const double ang0 = (a.mode == 0) ? static_cast<double>(jc) * omega_corr(pr)
+                                              : static_cast<double>(jc / G - jc) * a.omega[pr];
             angle_cos_sin(ang0, c[hk], sn[hk]);
           }
 #pragma unroll
@@ -161,7 +182,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
               *reinterpret_cast<float2*>(cs + (8 * hk + kk) * CS_STRIDE + pr * 8) = make_float2(c[hk], sn[hk]);
               float dc = fi_c[e], ds = fi_s[e];
               if (a.mode != 0) {
-                const bool stay = ((j0 + 8 * hk + kk + 1) % a.G) == 0;
+                const bool stay = ((j0 + 8 * hk + kk + 1) % G) == 0;
                 dc = stay ? 1.f : pa_c[e];
                 ds = stay ? 0.f : pa_s[e];
               }
@@ -188,8 +209,8 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   uint32_t qa_o[KC][2], qa_l[KC][2];
   {
     const bool row_ok = g8 < g;
-    const __nv_bfloat16* qrow = a.q + static_cast<long long>(kvh * g + (row_ok ? g8 : 0)) * D;
-    const double pl = (a.mode == 0) ? static_cast<double>(p) : static_cast<double>(p / a.G);
+    const __nv_bfloat16* qrow = a.q + (static_cast<long long>(bz) * a.hq + kvh * g + (row_ok ? g8 : 0)) * D;
+    const double pl = (a.mode == 0) ? static_cast<double>(p) : static_cast<double>(p / G);
 #pragma unroll
     for (int kc = 0; kc < KCP; ++kc)
 #pragma unroll
@@ -208,7 +229,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
           xo[e] = x * c - y * sn;
           yo[e] = y * c + x * sn;
           if (a.mode == 0)
-            angle_cos_sin(pl * a.omega_long[d + e], c, sn);
+            angle_cos_sin(pl * omega_long(d + e), c, sn);
           else
             angle_cos_sin(pl * a.omega[d + e], c, sn);
           xl[e] = x * c - y * sn;
@@ -305,6 +326,20 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
       o[mt][2] *= al0;
       o[mt][3] *= al1;
     }
+    // Keys past the split's end (the last stage of a split, warp-uniform) have P = 0, but 0 * NaN
+    // is NaN: their V rows hold whatever the cache (or a paged pool's slot) held, so this warp
+    // zeroes its own rows of them before the PV products read them.
+    const bool ragged = jt + 7 >= jend;
+    if (ragged) {
+      uint8_t* vrows = sV + st * STAGE_KV + hl * HALVES * HEAD_TILE;
+#pragma unroll 1
+      for (int r = 0; r < 8; ++r)
+        if (jt + r >= jend && lane < 8)
+#pragma unroll
+          for (int hf = 0; hf < HALVES; ++hf)
+            *reinterpret_cast<uint4*>(vrows + hf * HEAD_TILE + (nt * 8 + r) * 128 + lane * 16) = make_uint4(0, 0, 0, 0);
+      __syncwarp();
+    }
 #pragma unroll
     for (int mt = 0; mt < MT; mt += 2) {
       // A = V^T: four 8x8 blocks (keys x d) of d-blocks 2mt .. 2mt+3, transposed by ldmatrix
@@ -314,6 +349,8 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
       mma_bf16_1688(o[mt], r[0], r[1], pb);
       mma_bf16_1688(o[mt + 1], r[2], r[3], pb);
     }
+    // the zeroes above are generic-proxy writes to a slot the next TMA fill overwrites
+    if (ragged) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
   }
@@ -321,7 +358,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   // partial results of this warp (its own split): rows < g
   l_r += __shfl_xor_sync(0xffffffffu, l_r, 1);
   l_r += __shfl_xor_sync(0xffffffffu, l_r, 2);
-  const long long split = static_cast<long long>(blockIdx.x) * 2 + nt;
+  const long long split = static_cast<long long>(bz) * a.parts_stride + static_cast<long long>(blockIdx.x) * 2 + nt;
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int row = 2 * t4 + e;
@@ -358,14 +395,26 @@ constexpr int decode_threads() {
 // strided share of the partials, one lane per dimension, and shared memory adds the warps.
 constexpr int COMBINE_WARPS = 8;
 
+// Batched (grid.z = sequence, seq_lens non-null): sequence b's partials start at row
+// b * parts_stride, and only the 2 * ceil(seq_lens[b] / split_len) of its splits that hold keys
+// were written; out / lse advance by hq rows per sequence.
 template <int D>
 __global__ void __launch_bounds__(32 * COMBINE_WARPS) decode_combine_kernel(
     const float* __restrict__ part_o, const float* __restrict__ part_ml, int n_split, int hq,
-    __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+    __nv_bfloat16* __restrict__ out, float* __restrict__ lse, const int* __restrict__ seq_lens, int split_len,
+    int parts_stride) {
   __shared__ float red_acc[COMBINE_WARPS][32];
   __shared__ float red_l[COMBINE_WARPS];
   __shared__ float warp_max[COMBINE_WARPS];
   pdl_wait();  // the partials of the previous kernel are complete and visible
+  const int b = blockIdx.z;
+  if (seq_lens) {
+    n_split = 2 * ((seq_lens[b] + split_len - 1) / split_len);
+    part_o += static_cast<long long>(b) * parts_stride * hq * D;
+    part_ml += static_cast<long long>(b) * parts_stride * hq * 2;
+    out += static_cast<long long>(b) * hq * D;
+    if (lse) lse += static_cast<long long>(b) * hq;
+  }
   const int h = blockIdx.x, d = 32 * blockIdx.y + (threadIdx.x & 31);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // global max of the partial maxima
@@ -413,24 +462,34 @@ struct AppendArgs {
   __nv_bfloat16* vcache;
   int hkv, p;
   double omega[64];
+  // batched paged form (grid.y = sequence): position seq_lens[b] - 1, pool row via the block table
+  const int* seq_lens;
+  const int* block_table;
+  int max_pages, page_size;
 };
 
 template <int D>
 __global__ void decode_append_kernel(const __grid_constant__ AppendArgs a) {
   constexpr int P = D / 2;
   pdl_launch_dependents();  // the partial kernel may start; only its stage holding row p waits for us
-  const int h = blockIdx.x, lane = threadIdx.x;
-  const __nv_bfloat16* kr = a.k_new + h * D;
-  __nv_bfloat16* kd = a.kcache + (static_cast<long long>(a.p) * a.hkv + h) * D;
+  const int h = blockIdx.x, lane = threadIdx.x, b = blockIdx.y;
+  const bool paged = a.seq_lens != nullptr;
+  const int p = paged ? a.seq_lens[b] - 1 : a.p;  // logical position of the new token
+  const long long row =
+      paged ? static_cast<long long>(a.block_table[static_cast<long long>(b) * a.max_pages + p / a.page_size]) *
+                      a.page_size + p % a.page_size
+            : p;
+  const __nv_bfloat16* kr = a.k_new + (static_cast<long long>(b) * a.hkv + h) * D;
+  __nv_bfloat16* kd = a.kcache + (row * a.hkv + h) * D;
   for (int pr = lane; pr < P; pr += 32) {
     float c, s;
-    angle_cos_sin(static_cast<double>(a.p) * a.omega[pr], c, s);
+    angle_cos_sin(static_cast<double>(p) * a.omega[pr], c, s);
     const float x = __bfloat162float(kr[pr]), y = __bfloat162float(kr[pr + P]);
     kd[pr] = __float2bfloat16(x * c - y * s);
     kd[pr + P] = __float2bfloat16(y * c + x * s);
   }
-  const __nv_bfloat16* vr = a.v_new + h * D;
-  __nv_bfloat16* vd = a.vcache + (static_cast<long long>(a.p) * a.hkv + h) * D;
+  const __nv_bfloat16* vr = a.v_new + (static_cast<long long>(b) * a.hkv + h) * D;
+  __nv_bfloat16* vd = a.vcache + (row * a.hkv + h) * D;
   for (int d = lane; d < D; d += 32) vd[d] = vr[d];
 }
 

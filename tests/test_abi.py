@@ -188,6 +188,24 @@ def test_qknorm_validation_before_launch(lib):
     assert call(params()) == 5               # valid: stops at the (empty) workspace
 
 
+def test_paged_decode_validation_before_launch(lib):
+    f = lib.bifocal_decode_paged
+
+    def call(p, pages=100, page=32, table=FAKE, max_pages=10, lens=FAKE, max_len=300, batch=2, ws=FAKE, wsb=0):
+        return f(FAKE, FAKE, FAKE, FAKE, FAKE, pages, page, table, max_pages, lens, max_len, batch, ctypes.byref(p),
+                 FAKE, None, ws, wsb, None)
+
+    assert call(params(), table=None) == 1
+    assert call(params(), lens=None) == 1
+    assert call(params(), batch=0) == 1
+    assert call(params(), page=24) == 1          # not a multiple of 16
+    assert call(params(), max_pages=9) == 1      # 9 * 32 < 300
+    assert call(params(flags=bfl.FLAG_WINDOW)) == 2
+    assert call(params()) == 5                   # valid: stops at the (empty) workspace
+    assert bfl.decode_paged_workspace_size(2, 300, params()) > 0
+    assert bfl.decode_paged_workspace_size(0, 300, params()) == 0
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     mod = importlib.import_module("rope_context_extension_bifocal_b200")
