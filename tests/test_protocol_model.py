@@ -1,0 +1,238 @@
+"""A model of the ping-pong prefill kernel's barrier protocol, run under random interleavings (CPU).
+
+The kernel (csrc/prefill_tc2.cuh) has five actors per CTA: a TMA producer, the MMA issuer, the
+tensor pipe that executes the issued MMAs in order, and two softmax groups (tiles A and B). They
+meet on mbarriers that are waited on by phase parity. The model replays each actor's program
+step by step in a random order and checks that
+- no actor ever passes a parity wait on the wrong phase (a parity alias: the barrier ran two
+  phases ahead of the waiter),
+- the producer never overwrites Q while a QK^T that reads it is pending,
+- every program finishes (no deadlock),
+for the visit schedules of every kernel kind: plain, bifocal (long visits, Q reload, local visits),
+sliding window (long visits skipped), and query tiles at offsets that are not tile multiples
+(chunked prefill). The schedule below restates the kernel's tile classification.
+"""
+import random
+
+import pytest
+
+BM = BN = 128
+NSLOT = 4  # K/V ring slots: two per visit (K, then V)
+
+
+def schedule(i0, n_kt, w0, kind):
+    """Visit counts of one query tile starting at absolute row i0 with n_kt key tiles."""
+    if kind == "plain":
+        return dict(n_long=0, n_loc=n_kt)
+    A = (i0 - (BN - 1) - w0) // BN        # tiles t <= A: every pair long-range
+    C = (i0 + (BM - 1) - w0) // BN + 1    # tiles t >= C: every pair local
+    n_lf = min(max(A + 1, 0), n_kt)
+    n_b = max(min(C, n_kt) - n_lf, 0)
+    n_bl = n_b if w0 > 0 else 0
+    n_of = n_kt - n_lf - n_b
+    if kind == "window":
+        return dict(n_long=0, n_loc=n_bl + n_of)
+    return dict(n_long=n_lf + n_b, n_loc=n_bl + n_of)
+
+
+class Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.tx, self.phase = count, count, 0, 0
+
+    def arrive(self):
+        self.pending -= 1
+        self._flip()
+
+    def expect(self, n):
+        self.tx += n
+        self.pending -= 1
+        self._flip()
+
+    def complete_tx(self, n):
+        self.tx -= n
+        self._flip()
+
+    def _flip(self):
+        if self.pending == 0 and self.tx == 0:
+            self.phase += 1
+            self.pending = self.count
+
+    def passed(self, parity):  # try_wait.parity: true once the phase with this parity completed
+        return (self.phase & 1) != parity
+
+
+def run_protocol(sch, rnd, skip_q_free_wait=False):
+    nv = sch["n_long"] + sch["n_loc"]
+    has_long, has_orig = sch["n_long"] > 0, sch["n_loc"] > 0
+    reload_q = has_long and has_orig
+    v_sw = sch["n_long"]
+    full = [Bar(1) for _ in range(NSLOT)]
+    empty = [Bar(1) for _ in range(NSLOT)]
+    s_full, p_ready, o_done = [Bar(1), Bar(1)], [Bar(4), Bar(4)], [Bar(1), Bar(1)]
+    q_full, q_free = Bar(1), Bar(1)
+    tma, pipe = [], []
+    state = {"q_readers": 0}
+
+    prod = [("loadq",)]
+    n = 0
+    for v in range(nv):
+        if reload_q and v == v_sw:
+            prod += ([] if skip_q_free_wait else [("wait", q_free, 0)]) + [("loadq",)]
+        for _ in range(2):
+            prod.append(("fill", n))
+            n += 1
+
+    mma = [("wait", q_full, 0), ("wait", full[0], 0), ("qk", 0), ("qk", 1), ("commit", empty[0])]
+    if reload_q and v_sw == 1:
+        mma.append(("commit", q_free))
+    for v in range(nv):
+        vs = (2 * v + 1) % NSLOT
+        mma += [("wait", p_ready[0], v & 1), ("wait", full[vs], ((2 * v + 1) // NSLOT) & 1), ("pv", 0)]
+        more = v + 1 < nv
+        if more:
+            if reload_q and v + 1 == v_sw:
+                mma.append(("wait", q_full, 1))
+            k2 = (2 * (v + 1)) % NSLOT
+            mma += [("wait", full[k2], ((2 * (v + 1)) // NSLOT) & 1), ("qk", 0)]
+        mma += [("wait", p_ready[1], v & 1), ("pv", 1), ("commit", empty[vs])]
+        if more:
+            mma += [("qk", 1), ("commit", empty[(2 * (v + 1)) % NSLOT])]
+            if reload_q and v + 2 == v_sw:
+                mma.append(("commit", q_free))
+
+    def softmax_prog(x):
+        prog = []
+        for v in range(nv):
+            prog.append(("wait_s", x, v))
+            if v >= 1:
+                prog.append(("wait_o", x, v - 1))
+            prog.append(("arrive", x))
+        if nv:
+            prog.append(("wait_o", x, nv - 1))
+        return prog
+
+    progs = {"prod": prod, "mma": mma, "smA": softmax_prog(0), "smB": softmax_prog(1)}
+    pc = {k: 0 for k in progs}
+
+    def step_prod():
+        st = progs["prod"][pc["prod"]]
+        if st[0] == "loadq":
+            assert state["q_readers"] == 0, "Q overwritten while a QK^T reads it"
+            q_full.expect(1)
+            tma.append(q_full)
+        elif st[0] == "wait":
+            if not st[1].passed(st[2]):
+                return False
+        else:
+            k = st[1]
+            s, use = k % NSLOT, k // NSLOT
+            if use > 0:
+                if not empty[s].passed((use - 1) & 1):
+                    return False
+                assert empty[s].phase == use, "empty-slot parity alias"
+            full[s].expect(1)
+            tma.append(full[s])
+        return True
+
+    def step_mma():
+        st = progs["mma"][pc["mma"]]
+        if st[0] == "wait":
+            return st[1].passed(st[2])
+        if st[0] == "qk":
+            state["q_readers"] += 1
+            pipe.append(("s_full", st[1]))
+        elif st[0] == "pv":
+            pipe.append(("o_done", st[1]))
+        else:
+            pipe.append(("bar", st[1]))
+        return True
+
+    def step_tensor():
+        kind, arg = pipe.pop(0)
+        if kind == "s_full":
+            state["q_readers"] -= 1
+            s_full[arg].arrive()
+        elif kind == "o_done":
+            o_done[arg].arrive()
+        else:
+            arg.arrive()
+        return True
+
+    def step_softmax(name, x):
+        st = progs[name][pc[name]]
+        if st[0] == "wait_s":
+            if not s_full[x].passed(st[2] & 1):
+                return False
+            assert s_full[x].phase == st[2] + 1, "S parity alias"
+        elif st[0] == "wait_o":
+            if not o_done[x].passed(st[2] & 1):
+                return False
+            assert o_done[x].phase >= st[2] + 1, "O parity alias"
+        else:
+            for _ in range(4):
+                p_ready[x].arrive()
+        return True
+
+    def actors():
+        out = []
+        if pc["prod"] < len(progs["prod"]):
+            out.append(("prod", step_prod))
+        if tma:
+            out.append(("tma", lambda: (tma.pop(rnd.randrange(len(tma))).complete_tx(1), True)[1]))
+        if pc["mma"] < len(progs["mma"]):
+            out.append(("mma", step_mma))
+        if pipe:
+            out.append(("tensor", step_tensor))
+        for name, x in (("smA", 0), ("smB", 1)):
+            if pc[name] < len(progs[name]):
+                out.append((name, lambda name=name, x=x: step_softmax(name, x)))
+        return out
+
+    while True:
+        acts = actors()
+        if not acts:
+            return True
+        rnd.shuffle(acts)
+        for name, fn in acts:
+            if fn():
+                if name in pc:
+                    pc[name] += 1
+                break
+        else:
+            raise AssertionError(f"deadlock at {pc}")
+
+
+CASES = [
+    # (L queries, q_off, w0, kind)
+    (1100, 0, 300, "bifocal"), (4096, 0, 0, "bifocal"), (4096, 0, 1, "bifocal"), (3000, 0, 5000, "bifocal"),
+    (8192, 0, 127, "bifocal"), (8192, 0, 128, "bifocal"), (2048, 0, 0, "plain"),
+    (2048, 0, 512, "window"), (2048, 0, 1000, "window"), (4096, 0, 129, "window"),
+    (300, 1000, 100, "bifocal"), (333, 777, 50, "bifocal"), (300, 1024, 64, "window"),
+]
+
+
+@pytest.mark.parametrize("Lq,q_off,w0,kind", CASES)
+def test_protocol_completes_without_aliasing(Lq, q_off, w0, kind):
+    rnd = random.Random(Lq * 31 + q_off + w0)
+    n_qt = (Lq + BM - 1) // BM
+    for qt in range(n_qt):
+        i0 = q_off + qt * BM
+        n_kt = (min(i0 + BM, q_off + Lq) + BN - 1) // BN
+        sch = schedule(i0, n_kt, w0, kind)
+        for _ in range(2):
+            assert run_protocol(sch, rnd) is True
+
+
+def test_model_catches_a_missing_q_free_wait():
+    # planted protocol mistake: the producer reloads Q without waiting for q_free, so in some
+    # interleavings the original-RoPE Q lands while a long-range QK^T still reads the old one
+    sch = schedule(2048, 17, 300, "bifocal")
+    assert sch["n_long"] > 0 and sch["n_loc"] > 0
+    rnd = random.Random(7)
+    caught = 0
+    for _ in range(200):
+        try:
+            run_protocol(sch, rnd, skip_q_free_wait=True)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
