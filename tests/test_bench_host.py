@@ -11,9 +11,15 @@ if ROOT not in sys.path:
 import bench  # noqa: E402
 
 
-def test_traffic_reported_for_the_captured_sources():
+def test_traffic_follows_the_source_hash():
+    import hashlib
     t = bench.TRAFFIC["prefill_attention"]
-    assert bench.measured_traffic("prefill_attention") == t["bytes_per_launch"]
+    h = hashlib.sha256()
+    for f in t["sources"]:
+        with open(os.path.join(ROOT, "rope_context_extension_bifocal_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    want = t["bytes_per_launch"] if h.hexdigest() == t["sha256"] else None
+    assert bench.measured_traffic("prefill_attention") == want
 
 
 def test_traffic_null_once_the_kernel_changes(monkeypatch):
