@@ -33,15 +33,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel,
-# from one single-pass ncu capture of a full-size launch (the command is in the profile named
-# below), keyed by the SHA-256 of the kernel's sources at capture time: when the sources no
-# longer match, the kernel has changed since the counters were taken and traffic is null.
+# from one single-pass ncu capture of a full-size launch, keyed by the SHA-256 of the kernel's
+# sources at capture time: when the sources no longer match, the kernel has changed since the
+# counters were taken and traffic is null.
 TRAFFIC = {
     "prefill_attention": {
         "bytes_per_launch": 60.62e9 + 1.11e9,
         "sources": ["common.cuh", "prefill_tc.cuh", "prefill_tc2.cuh"],
         "sha256": "b5d7f2e31ad8806c5666de6ea4e04cfb217ab0415fab212aa6554ff7b5b692fb",
-        "profile": "profiles/attn_tc2_traffic_L131072.md",
     },
 }
 
@@ -217,6 +216,45 @@ def oracle_sample(q, k, v, w, rows, heads):
     return dt, flops
 
 
+def cpu_baseline_measure(q, k, v, w):
+    """The fp64 oracle on a bounded sample of the prefill workload, on the host cores, with the
+    rate it reached and, labelled as extrapolated, the time it would take for the 512-row-per-head
+    sample of the parity tests and for the whole prefill (cost per row = its causal key count),
+    plus the decode oracle's seconds per step at the decode workload's length."""
+    import numpy as np
+
+    import oracle.bifocal_ref as R
+    import seeded_inputs as si
+    rows512 = si.sample_rows(w.seed, w.L, w.w0, w.w_pretrained, 512)
+    rows = rows512[::43]  # 12 rows spread over the sequence, both branches over all their keys
+    dt, fl = oracle_sample(q, k, v, w, [int(r) for r in rows], list(range(w.hq)))
+    keys = float(sum(int(r) + 1 for r in rows)) * w.hq
+    rate = keys / dt
+    out = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "kind": "oracle",
+           "sample": f"query rows {', '.join(str(int(r)) for r in rows)} (every 43rd row of the 512-row parity "
+                     f"sample) x all {w.hq} heads of the same workload, fp64 NumPy, {dt:.1f} s",
+           "sample_s": dt, "rows_per_s": len(rows) * w.hq / dt, "causal_keys_per_s": rate,
+           "extrapolated_512_row_sample_s": float(sum(int(r) + 1 for r in rows512)) * w.hq / rate,
+           "extrapolated_full_prefill_s": w.L * (w.L + 1) / 2.0 * w.hq / rate}
+    # decode: the oracle's step at the decode workload's length (cache 131000 + 1), one step timed
+    dw = si.DECODE_128K
+    stream = si.DecodeStream(dw)
+    kp, vp = stream.cache_prefix()
+    qd, kn, vn = stream.step()
+    L = dw.prefix_len + 1
+    kc = np.zeros((L, dw.hkv, dw.head_dim))
+    vc = np.zeros((L, dw.hkv, dw.head_dim))
+    kc[:L - 1] = kp.float().double().numpy()
+    vc[:L - 1] = vp.float().double().numpy()
+    kc[L - 1] = R.rope_keys_for_cache(kn[None].float().double().numpy(), dw.theta, start=L - 1)[0]
+    vc[L - 1] = vn.float().double().numpy()
+    t0 = time.perf_counter()
+    R.bifocal_decode_reference(qd.float().double().numpy(), kc, vc, L, dw.w0, dw.w_pretrained, dw.theta, dw.mode)
+    out["decode_s_per_step"] = time.perf_counter() - t0
+    out["decode_note"] = f"bifocal_decode_reference at L = {L}, Hq {dw.hq}, Hkv {dw.hkv}, one step"
+    return out
+
+
 # ------------------------------------------------------------------ reference arm
 def run_reference(args):
     """The fp64 CPU oracle as the reference arm, on bounded samples of the same workload."""
@@ -318,6 +356,23 @@ def run_ours(args):
                 "traffic_unit": "bytes per launch (DRAM read + write, ncu)", "kernel": "bifocal attention (prefill)",
                 "peak_kind": f"{peak_kind} bf16 dense burst", "kernel_ms": attn_ms, "rope_pass_ms": rope_ms}
 
+    # ---- the fused-load kernel (RoPE and correction inside the tile loads, no workspace): A/B
+    fused = None
+    if not args.no_fused:
+        pf = bfl.make_params(w.hq, w.hkv, w.head_dim, w.w0, w.w_pretrained, w.theta, w.mode, None,
+                             bfl.FLAG_FUSED_ROPE)
+
+        def step_fused():
+            bfl._prefill("bifocal_prefill", q, k, v, pf, True, False, out, ws, None)
+
+        n_f = max(3, args.steps)
+        f_ms = time_loop(step_fused, n_f, 1, dist, torch) / n_f
+        f_t = flops / (f_ms / 1e3) / 1e12
+        fused = {"ms": f_ms, "tflops": f_t, "frac_of_peak": f_t / peak_t, "steps": n_f,
+                 "vs_rope_pass_step": ms_per_step / f_ms,
+                 "note": "bifocal_prefill with BF_FLAG_FUSED_ROPE: one launch, raw q/k tiles rotated in shared "
+                         "memory, empty workspace (the headline step is RoPE pass + attention)"}
+
     # ---- plain comparator (same shapes, original RoPE only)
     def step_plain():
         bfl.rope_causal_prefill(q, k, v, theta=w.theta, out=out, workspace=ws)
@@ -374,19 +429,28 @@ def run_ours(args):
         qc, kc_, vc_ = q[0, P0:], k[0, P0:], v[0, P0:]
         outc = torch.empty(C, w.hq, w.head_dim, dtype=torch.bfloat16, device=dev)
 
-        def step_chunk():
+        def step_chunk(flags=0):
             bfl.bifocal_prefill_chunk(qc, kc_, vc_, kc_all, vc_all, P0, w0=w.w0, w_pretrained=w.w_pretrained,
-                                      theta=w.theta, mode=w.mode, want_lse=False, out=outc, workspace=wsc)
+                                      theta=w.theta, mode=w.mode, want_lse=False, out=outc, workspace=wsc,
+                                      flags=flags)
 
         n_chunk = max(3, args.steps)
         chunk_ms = time_loop(step_chunk, n_chunk, 1, dist, torch) / n_chunk
         chunk_flops = 4.0 * w.head_dim * w.hq * (C * P0 + C * (C + 1) / 2)
         chunk_tflops = chunk_flops / (chunk_ms / 1e3) / 1e12
+        fchunk_ms = time_loop(lambda: step_chunk(bfl.FLAG_FUSED_ROPE), n_chunk, 1, dist, torch) / n_chunk
+        fchunk_tflops = chunk_flops / (fchunk_ms / 1e3) / 1e12
+        pfc = bfl.make_params(w.hq, w.hkv, w.head_dim, w.w0, w.w_pretrained, w.theta, w.mode, None,
+                              bfl.FLAG_FUSED_ROPE)
         chunk = {"workload": f"qwen3_8b_chunk_after_{P0}_cached_C{C}_w{w.w0}", "P0": P0, "C": C,
                  "G": bfl.bifocal_factor(w.L, w.w_pretrained), "ms": chunk_ms, "tflops": chunk_tflops,
-                 "frac_of_peak": chunk_tflops / peak_t,
+                 "frac_of_peak": chunk_tflops / peak_t, "workspace_bytes": wsc.numel(),
                  "note": "one call = cache re-phase pass + chunk RoPE pass + attention (3 launches); "
-                         "FLOPs counted over the chunk's causal pairs"}
+                         "FLOPs counted over the chunk's causal pairs",
+                 "fused": {"ms": fchunk_ms, "tflops": fchunk_tflops, "frac_of_peak": fchunk_tflops / peak_t,
+                           "workspace_bytes": bfl.prefill_chunk_workspace_size(P0, C, pfc),
+                           "note": "BF_FLAG_FUSED_ROPE: chunk rows written to the cache, then one attention "
+                                   "launch that re-phases cached keys in its tile loads (2 launches)"}}
         del kc_all, vc_all, wsc, outc
 
     # ---- sliding-window prefill (the local layers of a hybrid model), window = w0
@@ -422,12 +486,10 @@ def run_ours(args):
     # ---- CPU baseline: the oracle on a bounded sample, rank 0, N = 1 only
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        rows = list(range(w.L - 8, w.L))
-        dt, fl = oracle_sample(q_h, k_h, v_h, w, rows, list(range(w.hq)))
         cores, threads = cpu_info()
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": f"query rows {rows[0]}-{rows[-1]} x all {w.hq} heads of the same workload "
-                         f"(fp64 NumPy, {dt:.1f} s; host has {cores} usable cores)"}
+        cpu = cpu_baseline_measure(q_h, k_h, v_h, w)
+        cpu["cores"] = threads
+        cpu["sample"] += f"; host has {cores} usable cores"
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": dist.world, "steps": args.steps,
@@ -444,6 +506,7 @@ def run_ours(args):
         "overhead_vs_plain": {"prefill": overhead_prefill, "prefill_plain_ms": plain_ms,
                               "decode": decode["overhead_vs_plain"] if decode else None},
         "w0_sweep": sweep,
+        "fused_prefill": fused,
         "decode": decode,
         "chunked_prefill": chunk,
         "window_prefill": window,
@@ -565,6 +628,65 @@ def run_paged(args, torch, bfl, si, dev, peaks, peak_kind):
             "G": [bfl.bifocal_factor(L, wp) for L in lens]}
 
 
+def run_case(args):
+    """One named case, `--reps` timed calls after an untimed one, on cuda:0 (for ncu captures and
+    quick timing). Inputs follow the seeded recipe (iid N(0,1) bf16)."""
+    import torch
+
+    import rope_context_extension_bifocal_b200 as bfl
+    import seeded_inputs as si
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    a = args
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if a.case.startswith("prefill"):
+        q, k, v = (t.to(dev) for t in si.random_qkv(3, 1, a.L, a.hq, a.hkv, a.D, "bf16"))
+        p = bfl.make_params(a.hq, a.hkv, a.D, a.w0, a.w_pretrained, a.theta, a.mode, None, a.flags)
+        ws = torch.empty(bfl.prefill_workspace_size(bfl.DTYPE_BF16, 1, a.L, p), dtype=torch.uint8, device=dev)
+        out = torch.empty(1, a.L, a.hq, a.D, dtype=torch.bfloat16, device=dev)
+
+        def call():
+            if a.case == "prefill":
+                bfl.bifocal_prefill(q, k, v, w0=a.w0, w_pretrained=a.w_pretrained, theta=a.theta, mode=a.mode,
+                                    flags=a.flags, out=out, workspace=ws)
+            else:
+                bfl.rope_causal_prefill(q, k, v, theta=a.theta, out=out, workspace=ws)
+        work, unit = 4.0 * a.L * a.L / 2 * a.D * a.hq, "TFLOP/s"
+    else:
+        cap = a.L + 16
+        kc = torch.randn(cap, a.hkv, a.D, device=dev).to(torch.bfloat16)
+        vc = torch.randn(cap, a.hkv, a.D, device=dev).to(torch.bfloat16)
+        q = torch.randn(a.hq, a.D, device=dev).to(torch.bfloat16)
+        kn = torch.randn(a.hkv, a.D, device=dev).to(torch.bfloat16)
+        vn = torch.randn(a.hkv, a.D, device=dev).to(torch.bfloat16)
+        p = bfl.make_params(a.hq, a.hkv, a.D, a.w0, a.w_pretrained, a.theta, a.mode, None, a.flags)
+        ws = torch.empty(bfl.decode_workspace_size(cap, p), dtype=torch.uint8, device=dev)
+        out = torch.empty(a.hq, a.D, dtype=torch.bfloat16, device=dev)
+
+        def call():
+            if a.case == "decode":
+                bfl.bifocal_decode(q, kn, vn, kc, vc, a.L, w0=a.w0, w_pretrained=a.w_pretrained, theta=a.theta,
+                                   mode=a.mode, flags=a.flags, out=out, workspace=ws)
+            else:
+                bfl.rope_causal_decode(q, kn, vn, kc, vc, a.L, theta=a.theta, out=out, workspace=ws)
+        work, unit = 2.0 * 2 * a.L * a.hkv * a.D, "GB/s"  # cache bytes read
+    call()
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(a.reps):
+        call()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / a.reps
+    word = bfl.device_status_word()
+    rate = work / (ms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    print(json.dumps({"case": a.case, "L": a.L, "hq": a.hq, "hkv": a.hkv, "D": a.D, "w0": a.w0,
+                      "w_pretrained": a.w_pretrained, "ms_per_call": ms, "rate": rate, "unit": unit,
+                      "status_word": word}), flush=True)
+    return 0 if word == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -579,8 +701,22 @@ def main():
     ap.add_argument("--no-paged", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-fused", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    g = ap.add_argument_group("single case (--case): one kernel path timed alone, e.g. for an ncu capture")
+    g.add_argument("--case", choices=["prefill", "prefill_plain", "decode", "decode_plain"])
+    g.add_argument("--L", type=int, default=32768)
+    g.add_argument("--hq", type=int, default=32)
+    g.add_argument("--hkv", type=int, default=8)
+    g.add_argument("--D", type=int, default=128)
+    g.add_argument("--w-pretrained", type=int, default=8192)
+    g.add_argument("--theta", type=float, default=1e6)
+    g.add_argument("--mode", default="freq_interp", choices=["freq_interp", "pos_alias"])
+    g.add_argument("--reps", type=int, default=3)
+    g.add_argument("--flags", type=int, default=0, help="BF_FLAG_* bits")
     args = ap.parse_args()
+    if args.case:
+        return run_case(args)
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)

@@ -35,7 +35,8 @@
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
  *   - Errors: argument errors return BF_ERR_INVALID / BF_ERR_UNSUPPORTED / BF_ERR_WORKSPACE
  *     before any launch; a failed launch returns BF_ERR_CUDA. No call traps, aborts or prints.
- *     Device-side bounded waits that expire set a device status word, read (and cleared)
+ *     Device-side events the kernels cannot turn into a correct result (a bounded wait that
+ *     expires, an fp16 operand out of range) set a device status word, read (and cleared)
  *     by bifocal_last_device_error().
  */
 #ifndef BIFOCAL_H_
@@ -61,16 +62,28 @@ typedef enum {
   BF_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
   BF_ERR_TIMEOUT = 4,      /* a device-side bounded wait expired (reported by bifocal_last_device_error) */
   BF_ERR_WORKSPACE = 5,    /* workspace missing, misaligned or smaller than *_workspace_size */
-  BF_ERR_NO_DEVICE = 6     /* no CUDA device, or the device is not sm_100 */
+  BF_ERR_NO_DEVICE = 6,    /* no CUDA device, or the device is not sm_100 */
+  BF_ERR_RANGE = 7         /* an fp16 QK^T operand (a rotated query or key) was not finite once rounded to
+                              fp16 (|x| >= 65520, inf or NaN), so the result is not trustworthy (reported by
+                              bifocal_last_device_error) */
 } bf_status_t;
 
 typedef enum { BF_MODE_FREQ_INTERP = 0, BF_MODE_POS_ALIAS = 1 } bf_mode_t;
 typedef enum { BF_DTYPE_BF16 = 0, BF_DTYPE_FP32 = 1 } bf_dtype_t;
 
 /* flags */
-#define BF_FLAG_FORCE_BIFOCAL 1 /* run the two-branch kernel even when G == 1 or w0 >= L (results are equal) */
+#define BF_FLAG_FORCE_BIFOCAL 1 /* run the two-branch kernel even when G == 1 or w0 >= L (results are equal);
+                                   taken by every prefill, chunk and decode entry point alike */
 #define BF_FLAG_MMA_SYNC 2      /* prefill, D = 128: use the warp-level mma.sync kernel instead of tcgen05
                                    (comparison only; D = 64 always uses it) */
+#define BF_FLAG_FUSED_ROPE 8    /* prefill and chunk, bf16 inputs, head_dim 128, even GQA group: apply RoPE and
+                                 * the correction rotation inside the attention kernel's tile loads ([AF] module 3,
+                                 * on-the-fly rotation): the kernel reads raw q, raw k (prefill) or the cached
+                                 * original-RoPE keys (chunk) and forms each fp16 operand tile in shared memory,
+                                 * so the workspace is empty (*_workspace_size returns 0) and no rotated copy of
+                                 * q or k is written. bifocal_prefill_rope then only writes the cache rows asked
+                                 * for, and bifocal_prefill_attention returns BF_ERR_UNSUPPORTED (the kernel needs
+                                 * q and k: use bifocal_prefill). Other shapes and fp32 inputs ignore the flag. */
 #define BF_FLAG_WINDOW 4        /* sliding-window attention, the local layers of a hybrid model (Jet-Nemotron,
                                  * [AF] 影响): keep only pairs with 0 <= i - j < w0, under the original RoPE;
                                  * the long-range branch is dropped and G plays no part. Taken by
@@ -95,7 +108,7 @@ typedef struct {
 BF_API int32_t bifocal_factor(int64_t L, int32_t w_pretrained);
 
 /* Bytes of device workspace bifocal_prefill / rope_causal_prefill need for these sizes and
- * this input dtype: the rotated query and key forms (bf16) and, for fp32 inputs, a bf16
+ * this input dtype: the rotated query and key forms (fp16) and, for fp32 inputs, a bf16
  * copy of v. Host only. Returns 0 on invalid arguments. */
 BF_API size_t bifocal_prefill_workspace_size(int32_t dtype, int32_t batch, int32_t L, const bf_params_t* p);
 
@@ -178,6 +191,37 @@ BF_API bf_status_t bifocal_prefill_chunk(const void* q, const void* k, const voi
                                          int32_t C, const bf_params_t* p, void* kcache, void* vcache, int32_t cap,
                                          void* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
+/* Chunked prefill for a batch of sequences over a paged cache (vLLM-style block tables), each
+ * sequence with its own cached length, chunk length and G = max(1, ceil((P0_b + C_b) / w_pretrained))
+ * ([AF] module 2: the factor follows each sequence's current length; [AF] 影响 / [VS] 3: the
+ * serving engines this is meant to plug into batch sequences over paged caches). Always the
+ * fused kernel: RoPE and the correction rotation of cached keys happen in its tile loads, so
+ * there is no workspace and no second key copy.
+ *   q [T, hq, D], k / v [T, hkv, D] raw bf16: the chunks packed one after another in batch order
+ *          (sequence b's rows start at sum of chunk_lens[0 .. b-1]); T = sum of chunk_lens
+ *   chunk_lens, cached_lens [batch] int32, HOST arrays: C_b >= 1 new rows at positions
+ *          P0_b .. P0_b + C_b - 1 after P0_b >= 0 cached ones
+ *   kpool, vpool [pool_pages * page_size, hkv, D] bf16: keys under the ORIGINAL RoPE; the chunk's
+ *          keys R_orig(p) k and values are written at their positions first
+ *   block_table [batch, max_pages] int32 (device): key j of sequence b is pool row
+ *          block_table[b * max_pages + j / page_size] * page_size + j % page_size
+ *   page_size: a multiple of 16 that divides 128 or is a multiple of 128
+ *   out [T, hq, D] bf16;  lse [hq, T] fp32 (may be NULL)
+ * Sequence b's rows equal bifocal_prefill_chunk on its own cache. Flags: BF_FLAG_WINDOW as for the
+ * chunk call; a sequence whose G is 1 or whose w0 >= its length runs the two-branch kernel (as with
+ * BF_FLAG_FORCE_BIFOCAL, identical result). Pool rows past a sequence's end are never scored:
+ * their key rows are zeroed in shared memory and their value rows too, whatever the pool holds.
+ * block_table entries are trusted: every page a sequence's first P0_b + C_b positions use must be
+ * a page of the pool.
+ * Errors: as bifocal_prefill_chunk; BF_ERR_INVALID also for batch < 1, a bad page_size, P0_b < 0,
+ * C_b < 1, P0_b + C_b > max_pages * page_size or NULL arrays; BF_ERR_UNSUPPORTED for batch > 64,
+ * head_dim != 128 or an odd GQA group. */
+BF_API bf_status_t bifocal_prefill_chunk_paged(const void* q, const void* k, const void* v, int32_t batch,
+                                               const int32_t* chunk_lens, const int32_t* cached_lens,
+                                               const bf_params_t* p, void* kpool, void* vpool, int32_t pool_pages,
+                                               int32_t page_size, const int32_t* block_table, int32_t max_pages,
+                                               void* out, float* lse, void* stream);
+
 /* Bytes of device workspace bifocal_decode / rope_causal_decode need for a cache of up to
  * L_max rows: the split-KV partial results (fp32). Host only. 0 on invalid arguments. */
 BF_API size_t bifocal_decode_workspace_size(int32_t L_max, const bf_params_t* p);
@@ -236,7 +280,9 @@ BF_API bf_status_t bifocal_decode_paged(const void* q, const void* k_new, const 
  * bifocal_decode_workspace_size(L, p) bytes of it (10.7 MB for 32 query heads of 128);
  * larger problems are rejected with BF_ERR_WORKSPACE before any launch.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- * with that device current; make that first call before any stream capture.
+ * with that device current; make that first call before any stream capture. The address is
+ * kept per device together with the id of the context it was read in; after a device reset
+ * (a new primary context) the next call looks it up again.
  * All calls share the one array and it keeps the last call's contents: nothing in it needs
  * to start at zero, but calls that overlap on the GPU (other streams, other threads) race
  * on it and must be serialised by the caller. Arguments and errors as bifocal_decode. */
@@ -253,13 +299,37 @@ BF_API bf_status_t rope_causal_decode(const void* q, const void* k_new, const vo
 /* Human-readable name of a status code (static string, never NULL). */
 BF_API const char* bifocal_status_string(int32_t status);
 
-/* Reads and clears the device status word that bounded waits set when they expire on the
- * current device. Synchronises `stream` first. Returns BF_OK, BF_ERR_TIMEOUT or BF_ERR_CUDA. */
+/* Reads and clears the device status word of the current device. The kernels set it, without
+ * trapping, for the first of these events since it was last cleared:
+ *   - a bounded wait expired (a producer never delivered, or a wait ran past the limit): BF_ERR_TIMEOUT;
+ *   - an fp16 QK^T operand (a query or key after RoPE or the correction rotation, or a cached
+ *     bf16 key converted to fp16) was not finite once rounded to fp16 (|x| >= 65520, inf or
+ *     NaN): BF_ERR_RANGE. The decode kernel detects it as a non-finite score of a valid key.
+ * Synchronises `stream` first. Returns BF_OK, BF_ERR_TIMEOUT, BF_ERR_RANGE or BF_ERR_CUDA. */
 BF_API bf_status_t bifocal_last_device_error(void* stream);
 
-/* The raw device status word (not cleared): 0, or 1 | (site << 8) for the first bounded wait
- * that expired, where `site` numbers the wait in the kernel source. Synchronises the device. */
+/* The raw device status word (not cleared): 0, or code | (site << 8) for the first event, where
+ * code is 1 (a bounded wait expired) or 2 (an fp16 operand out of range) and `site` numbers the
+ * wait or the check in the kernel source. Synchronises the device. Returns -1 on a CUDA error. */
 BF_API int32_t bifocal_device_status_word(void);
+
+/* Test-only fault injection for the failure-detection tests. Not needed by any caller of the
+ * attention entry points; everything is off unless a test turns it on.
+ *   kind BF_FAULT_NONE: every injection off.
+ *   kind BF_FAULT_PREFILL_SKIP_FILL: in the tcgen05 ping-pong prefill kernel, the producer of CTA 0
+ *        never issues K/V fill number `arg` (no expect_tx, no copy), so the MMA issuer's wait for
+ *        it can only expire: the CTA gives up, every role leaves through the normal teardown
+ *        (no copy in flight, tensor memory freed) and the status word reports the wait's site.
+ *   kind BF_FAULT_DECODE_SKIP_STAGE: in the split-KV decode kernel, the producer of CTA 0 never
+ *        issues stage `arg`; the consumer warps' wait for it expires likewise.
+ *   wait_limit_ns: the limit of every bounded wait in ns; 0 restores the default of 2 s. A wait
+ *        consults it only after 20 ms, so a smaller limit acts as 20 ms.
+ * Synchronises the device before and after setting the controls. Returns BF_ERR_INVALID for an
+ * unknown kind, a negative arg (with a fault kind) or a negative limit; BF_ERR_CUDA on a CUDA error. */
+#define BF_FAULT_NONE 0
+#define BF_FAULT_PREFILL_SKIP_FILL 1
+#define BF_FAULT_DECODE_SKIP_STAGE 2
+BF_API bf_status_t bifocal_test_set_fault(int32_t kind, int32_t arg, int64_t wait_limit_ns);
 
 /* Library build identification (static string): kernels compiled in and their target. */
 BF_API const char* bifocal_build_info(void);

@@ -14,9 +14,10 @@ import os
 from typing import Optional, Tuple
 
 __all__ = [
-    "BifocalError", "FREQ_INTERP", "POS_ALIAS", "FLAG_FORCE_BIFOCAL", "FLAG_MMA_SYNC", "FLAG_WINDOW", "Params", "lib", "lib_path",
-    "bifocal_factor", "bifocal_prefill", "bifocal_prefill_rope", "bifocal_prefill_attention", "rope_causal_prefill", "bifocal_decode", "bifocal_decode_noalloc", "rope_causal_decode",
-    "prefill_workspace_size", "decode_workspace_size", "last_device_error", "build_info",
+    "BifocalError", "FREQ_INTERP", "POS_ALIAS", "FLAG_FORCE_BIFOCAL", "FLAG_MMA_SYNC", "FLAG_WINDOW", "FLAG_FUSED_ROPE", "Params", "lib", "lib_path",
+    "bifocal_factor", "bifocal_prefill", "bifocal_prefill_rope", "bifocal_prefill_attention", "rope_causal_prefill", "bifocal_prefill_chunk_paged", "bifocal_decode", "bifocal_decode_noalloc", "rope_causal_decode",
+    "prefill_workspace_size", "decode_workspace_size", "last_device_error", "build_info", "test_set_fault",
+    "STATUS_TIMEOUT", "STATUS_RANGE", "FAULT_NONE", "FAULT_PREFILL_SKIP_FILL", "FAULT_DECODE_SKIP_STAGE",
 ]
 
 FREQ_INTERP = "freq_interp"
@@ -25,7 +26,10 @@ _MODES = {FREQ_INTERP: 0, POS_ALIAS: 1}
 FLAG_FORCE_BIFOCAL = 1
 FLAG_MMA_SYNC = 2
 FLAG_WINDOW = 4
+FLAG_FUSED_ROPE = 8
 DTYPE_BF16, DTYPE_FP32 = 0, 1
+STATUS_TIMEOUT, STATUS_RANGE = 4, 7
+FAULT_NONE, FAULT_PREFILL_SKIP_FILL, FAULT_DECODE_SKIP_STAGE = 0, 1, 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -88,12 +92,16 @@ def _lib() -> ctypes.CDLL:
         L.bifocal_decode_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, vp, i32, vp, i32, i32, pp, vp, vp, vp, sz,
                                            vp]
         L.bifocal_decode_paged.restype = i32
+        L.bifocal_prefill_chunk_paged.argtypes = [vp, vp, vp, i32, vp, vp, pp, vp, vp, i32, i32, vp, i32, vp, vp,
+                                                  vp]
+        L.bifocal_prefill_chunk_paged.restype = i32
         L.bifocal_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, pp, vp, vp, vp]
         L.bifocal_decode_noalloc.restype = i32
         L.bifocal_status_string.argtypes, L.bifocal_status_string.restype = [i32], ctypes.c_char_p
         L.bifocal_last_device_error.argtypes, L.bifocal_last_device_error.restype = [vp], i32
         L.bifocal_build_info.argtypes, L.bifocal_build_info.restype = [], ctypes.c_char_p
         L.bifocal_device_status_word.argtypes, L.bifocal_device_status_word.restype = [], i32
+        L.bifocal_test_set_fault.argtypes, L.bifocal_test_set_fault.restype = [i32, i32, i64], i32
         _LIB = L
     return _LIB
 
@@ -252,6 +260,32 @@ def bifocal_prefill_chunk(q, k, v, kcache, vcache, P0: int, *, w0: int, w_pretra
     return out, lse
 
 
+def bifocal_prefill_chunk_paged(q, k, v, chunk_lens, cached_lens, kpool, vpool, page_size: int, block_table, *,
+                                w0: int, w_pretrained: int, theta: float, mode: str = FREQ_INTERP,
+                                scale: Optional[float] = None, flags: int = 0, want_lse: bool = True, out=None,
+                                stream=None):
+    """Chunked prefill for a batch over a paged cache. q [T, Hq, D], k / v [T, Hkv, D] raw bf16, the
+    chunks packed in batch order; chunk_lens / cached_lens: Python ints per sequence; kpool / vpool
+    [pages * page_size, Hkv, D] bf16; block_table [B, max_pages] int32 on the device. Returns
+    (out [T, Hq, D] bf16, lse [Hq, T] fp32 or None)."""
+    import torch
+    T, hq, D = q.shape
+    B = len(chunk_lens)
+    if len(cached_lens) != B or sum(int(c) for c in chunk_lens) != T:
+        raise BifocalError(1, "bifocal_prefill_chunk_paged: chunk_lens must sum to the packed rows")
+    p = make_params(hq, k.shape[1], D, w0, w_pretrained, theta, mode, scale, flags)
+    out = torch.empty(T, hq, D, dtype=torch.bfloat16, device=q.device) if out is None else out
+    lse = torch.empty(hq, T, dtype=torch.float32, device=q.device) if want_lse else None
+    cl = (ctypes.c_int32 * B)(*[int(c) for c in chunk_lens])
+    pl = (ctypes.c_int32 * B)(*[int(c) for c in cached_lens])
+    st = _lib().bifocal_prefill_chunk_paged(_ptr(q), _ptr(k), _ptr(v), B, cl, pl, ctypes.byref(p), _ptr(kpool),
+                                            _ptr(vpool), kpool.shape[0] // page_size, int(page_size),
+                                            _ptr(block_table), block_table.shape[1], _ptr(out), _ptr(lse),
+                                            _stream(stream))
+    _check(st, "bifocal_prefill_chunk_paged")
+    return out, lse
+
+
 def _decode(fn_name, q, k_new, v_new, kcache, vcache, L, params, want_lse, out, workspace, stream):
     import torch
     hq, D = q.shape
@@ -334,5 +368,12 @@ def device_status_word() -> int:
 
 
 def last_device_error(stream=None) -> int:
-    """Status of device-side bounded waits since the last call (0 = none expired)."""
+    """Status of the device-side checks since the last call, then cleared: 0, STATUS_TIMEOUT (a
+    bounded wait expired) or STATUS_RANGE (an fp16 QK^T operand was out of range)."""
     return int(_lib().bifocal_last_device_error(_stream(stream)))
+
+
+def test_set_fault(kind: int = FAULT_NONE, arg: int = 0, wait_limit_ns: int = 0) -> None:
+    """Test-only fault injection (see bifocal_test_set_fault in include/bifocal.h); the default
+    arguments turn every injection off and restore the 2 s wait limit."""
+    _check(_lib().bifocal_test_set_fault(int(kind), int(arg), int(wait_limit_ns)), "bifocal_test_set_fault")

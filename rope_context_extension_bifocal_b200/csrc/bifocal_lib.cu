@@ -3,6 +3,7 @@
 // that the device status word is a single object.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -131,13 +132,13 @@ bool make_k_map(CUtensorMap* map, const void* base, int L, int rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// V [b][L][hkv][128] bf16, box (64, 1, 128, 1), 128B swizzle: one 128-byte row per key.
-bool make_v_map(CUtensorMap* map, const void* base, int L, int hkv, int batch) {
+// V [b][L][hkv][128] bf16, box (64, 1, box_rows, 1), 128B swizzle: one 128-byte row per key.
+bool make_v_map(CUtensorMap* map, const void* base, int L, int hkv, int batch, int box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(hkv), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(batch)};
   cuuint64_t strides[3] = {256, static_cast<cuuint64_t>(hkv) * 256, static_cast<cuuint64_t>(L) * hkv * 256};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -149,8 +150,17 @@ struct PrefillLayout {
   size_t qo, ql, ko, kl, vb, total;
 };
 
+bool tc2_path(const bf_params_t* p);
+
+// The fused-load path: RoPE and the correction rotation inside the ping-pong kernel's tile
+// loads (bf16 inputs, D = 128, even GQA group), selected by BF_FLAG_FUSED_ROPE.
+bool fused_path(const bf_params_t* p, int dtype) {
+  return (p->flags & BF_FLAG_FUSED_ROPE) && dtype == BF_DTYPE_BF16 && tc2_path(p);
+}
+
 PrefillLayout prefill_layout(int dtype, int batch, int L, const bf_params_t* p) {
   PrefillLayout w{};
+  if (fused_path(p, dtype)) return w;  // nothing to stage: every operand is formed in the kernel
   const size_t qbytes = align256(static_cast<size_t>(batch) * L * p->hq * p->head_dim * 2);
   const size_t kbytes = align256(static_cast<size_t>(batch) * L * p->hkv * p->head_dim * 2);
   w.qo = 0;
@@ -184,6 +194,7 @@ struct PrefillPlan {
   int D, G;
   bool bif;  // two-branch kernel (else every pair is local: the plain kernel gives the same result)
   int kind;  // tcgen05 ping-pong kernel: KIND_PLAIN, KIND_BIFOCAL or KIND_WINDOW
+  bool fused;  // RoPE in the kernel's tile loads (no rotated copies in the workspace)
   PrefillLayout lay;
   Rope rope;
 };
@@ -198,7 +209,9 @@ bf_status_t plan_prefill(bool bifocal_api, int32_t dtype, int32_t batch, int32_t
   if (window && p->w0 < 1) return BF_ERR_INVALID;
   if (window && !tc2_path(p)) return BF_ERR_UNSUPPORTED;
   plan->lay = prefill_layout(dtype, batch, L, p);
-  if (!workspace || !aligned(workspace, 256) || ws_bytes < plan->lay.total) return BF_ERR_WORKSPACE;
+  if (plan->lay.total > 0 && (!workspace || !aligned(workspace, 256) || ws_bytes < plan->lay.total))
+    return BF_ERR_WORKSPACE;
+  plan->fused = fused_path(p, dtype);
   plan->D = p->head_dim;
   plan->G = bifocal_api ? factor(L, p->w_pretrained) : 1;
   plan->bif = !window && bifocal_api && ((p->flags & BF_FLAG_FORCE_BIFOCAL) || (plan->G > 1 && p->w0 < L));
@@ -250,6 +263,13 @@ bf_status_t prefill_rope_impl(bool bifocal_api, const void* q, const void* k, co
   pa.q_norm_w = q_norm_w;
   pa.k_norm_w = k_norm_w;
   pa.norm_eps = norm_eps;
+  if (plan.fused) {
+    // the attention kernel forms every operand itself: this step only writes the cache rows asked for
+    if (!kcache_out && !vcache_out) return BF_OK;
+    pa.keys_only = 1;
+    pa.need_long = 0;
+    pa.Qo = pa.Ql = pa.Ko = pa.Kl = nullptr;
+  }
   const long long rows = static_cast<long long>(batch) * L;
   const dim3 pgrid(static_cast<unsigned>((rows + 7) / 8));
   if (dtype == BF_DTYPE_BF16) {
@@ -266,6 +286,52 @@ bf_status_t prefill_rope_impl(bool bifocal_api, const void* q, const void* k, co
   return cudaGetLastError() == cudaSuccess ? BF_OK : BF_ERR_CUDA;
 }
 
+template <bool FUSED>
+cudaError_t launch_tc2_t(int kind, const bf::Tc2Args& ta, long long n_cta, cudaStream_t st) {
+  constexpr int smem = bf::attn_tc2_smem_bytes(FUSED);
+  auto kern = kind == bf::tc2::KIND_BIFOCAL  ? bf::attn_tc2_kernel<bf::tc2::KIND_BIFOCAL, FUSED>
+              : kind == bf::tc2::KIND_WINDOW ? bf::attn_tc2_kernel<bf::tc2::KIND_WINDOW, FUSED>
+                                             : bf::attn_tc2_kernel<bf::tc2::KIND_PLAIN, FUSED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<static_cast<unsigned>(n_cta), bf::tc2::NTHREADS2, smem, st>>>(ta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc2(int kind, bool fused, const bf::Tc2Args& ta, long long n_cta, cudaStream_t st) {
+  return fused ? launch_tc2_t<true>(kind, ta, n_cta, st) : launch_tc2_t<false>(kind, ta, n_cta, st);
+}
+
+// The fused ping-pong attention over raw bf16 q [batch, Lq, hq, 128] (rows at absolute positions
+// q_off..) and a key source [batch, L, hkv, 128] (raw k, or the cache of original-RoPE keys)
+// with V [batch, L, hkv, 128].
+bf_status_t fused_attention(int kind, const void* q, const void* ksrc, bool cache, const void* v, int batch, int L,
+                            int q_off, int Lq, int G, const bf_params_t* p, const Rope& rope, void* out, float* lse,
+                            cudaStream_t st) {
+  bf::Tc2Args ta;
+  std::memset(&ta, 0, sizeof(ta));
+  if (!make_v_map(&ta.v_map, v, L, p->hkv, batch) || !make_v_map(&ta.qo_map, q, Lq, p->hq, batch) ||
+      !make_v_map(&ta.ko_map, ksrc, L, p->hkv, batch))
+    return BF_ERR_CUDA;
+  ta.out = static_cast<bf16*>(out);
+  ta.lse = lse;
+  ta.L = L;
+  ta.hq = p->hq;
+  ta.hkv = p->hkv;
+  ta.batch = batch;
+  ta.w0 = kind != bf::tc2::KIND_PLAIN ? p->w0 : L;
+  ta.q_off = q_off;
+  ta.Lq = Lq;
+  ta.scale_log2 = scale_log2(p);
+  ta.src.cache = cache ? 1 : 0;
+  ta.src.mode = p->mode;
+  ta.src.G = G;
+  std::memcpy(ta.src.omega, rope.omega, sizeof(ta.src.omega));
+  const long long n_cta = static_cast<long long>((Lq + bf::tc::BM - 1) / bf::tc::BM) * (p->hq / 2) * batch;
+  if (n_cta > 0x7fffffffLL) return BF_ERR_UNSUPPORTED;
+  return launch_tc2(kind, true, ta, n_cta, st) == cudaSuccess ? BF_OK : BF_ERR_CUDA;
+}
+
 bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtype, int32_t batch, int32_t L,
                                    const bf_params_t* p, void* out, float* lse, void* workspace, size_t ws_bytes,
                                    void* stream) {
@@ -277,6 +343,7 @@ bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtyp
     return BF_ERR_INVALID;
   s = plan_prefill(bifocal_api, dtype, batch, L, p, workspace, ws_bytes, &plan);
   if (s != BF_OK) return s;
+  if (plan.fused) return BF_ERR_UNSUPPORTED;  // the fused kernel reads q and k itself: use the one-call form
   const int D = plan.D;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -316,12 +383,12 @@ bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtyp
     ta.q_off = 0;
     ta.Lq = L;
     ta.scale_log2 = aa.scale_log2;
-    constexpr int smem = bf::attn_tc2_smem_bytes();
+      constexpr int smem = bf::attn_tc2_smem_bytes();
     const long long n_cta = static_cast<long long>((L + bf::tc::BM - 1) / bf::tc::BM) * (p->hq / 2) * batch;
     if (n_cta > 0x7fffffffLL) return BF_ERR_UNSUPPORTED;
-    auto kern = plan.kind == bf::tc2::KIND_BIFOCAL  ? bf::attn_tc2_kernel<bf::tc2::KIND_BIFOCAL>
-                : plan.kind == bf::tc2::KIND_WINDOW ? bf::attn_tc2_kernel<bf::tc2::KIND_WINDOW>
-                                               : bf::attn_tc2_kernel<bf::tc2::KIND_PLAIN>;
+    auto kern = plan.kind == bf::tc2::KIND_BIFOCAL  ? bf::attn_tc2_kernel<bf::tc2::KIND_BIFOCAL, false>
+                : plan.kind == bf::tc2::KIND_WINDOW ? bf::attn_tc2_kernel<bf::tc2::KIND_WINDOW, false>
+                                               : bf::attn_tc2_kernel<bf::tc2::KIND_PLAIN, false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess) {
       kern<<<static_cast<unsigned>(n_cta), bf::tc2::NTHREADS2, smem, st>>>(ta);
@@ -366,8 +433,9 @@ struct ChunkLayout {
   size_t qo, ql, ko, kl, total;
 };
 
-ChunkLayout chunk_layout(int P0, int C, const bf_params_t* p) {
+ChunkLayout chunk_layout(int P0, int C, const bf_params_t* p, int dtype) {
   ChunkLayout w{};
+  if (fused_path(p, dtype)) return w;  // cached keys are re-phased in the kernel's tile loads
   const size_t qbytes = align256(static_cast<size_t>(C) * p->hq * p->head_dim * 2);
   const size_t kbytes = align256((static_cast<size_t>(P0) + C) * p->hkv * p->head_dim * 2);
   w.qo = 0;
@@ -396,13 +464,37 @@ bf_status_t chunk_impl(const void* q, const void* k, const void* v, int32_t dtyp
   const int L = P0 + C;
   const bool window = (p->flags & BF_FLAG_WINDOW) != 0;
   if (window && p->w0 < 1) return BF_ERR_INVALID;
-  const ChunkLayout lay = chunk_layout(P0, C, p);
-  if (!workspace || !aligned(workspace, 256) || ws_bytes < lay.total) return BF_ERR_WORKSPACE;
+  const ChunkLayout lay = chunk_layout(P0, C, p, dtype);
+  if (lay.total > 0 && (!workspace || !aligned(workspace, 256) || ws_bytes < lay.total)) return BF_ERR_WORKSPACE;
   const int G = factor(L, p->w_pretrained);
   const bool bif = !window && ((p->flags & BF_FLAG_FORCE_BIFOCAL) || (G > 1 && p->w0 < L));
   const int kind = window ? (p->w0 < L ? bf::tc2::KIND_WINDOW : bf::tc2::KIND_PLAIN) : (bif ? bf::tc2::KIND_BIFOCAL : bf::tc2::KIND_PLAIN);
   const Rope rope = make_rope(p->rope_theta, D, G);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fused_path(p, dtype)) {
+    // 1. the chunk's keys (original RoPE, bf16) and values into cache rows P0 ..
+    bf::PrepassArgs pa{};
+    pa.q = q;
+    pa.k = k;
+    pa.v = v;
+    pa.batch = 1;
+    pa.L = C;
+    pa.pos0 = P0;
+    pa.Lk = L;
+    pa.Lc = cap;
+    pa.hq = p->hq;
+    pa.hkv = p->hkv;
+    pa.G = G;
+    pa.mode = p->mode;
+    pa.keys_only = 1;
+    pa.kcache = static_cast<bf16*>(kcache);
+    pa.vcache = static_cast<bf16*>(vcache);
+    std::memcpy(pa.omega, rope.omega, sizeof(pa.omega));
+    bf::rope_prepass_kernel<bf16, 128><<<static_cast<unsigned>((C + 7) / 8), 256, 0, st>>>(pa);
+    if (cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
+    // 2. the chunk's queries over all L cached keys, read as stored and re-phased in the tile loads
+    return fused_attention(kind, q, kcache, true, vcache, 1, L, P0, C, G, p, rope, out, lse, st);
+  }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   __half* Qo = reinterpret_cast<__half*>(ws + lay.qo);
   __half* Ql = reinterpret_cast<__half*>(ws + lay.ql);
@@ -478,9 +570,9 @@ bf_status_t chunk_impl(const void* q, const void* k, const void* v, int32_t dtyp
   ta.scale_log2 = scale_log2(p);
   constexpr int smem = bf::attn_tc2_smem_bytes();
   const long long n_cta = static_cast<long long>((C + bf::tc::BM - 1) / bf::tc::BM) * (p->hq / 2);
-  auto kern = kind == bf::tc2::KIND_BIFOCAL  ? bf::attn_tc2_kernel<bf::tc2::KIND_BIFOCAL>
-              : kind == bf::tc2::KIND_WINDOW ? bf::attn_tc2_kernel<bf::tc2::KIND_WINDOW>
-                                        : bf::attn_tc2_kernel<bf::tc2::KIND_PLAIN>;
+  auto kern = kind == bf::tc2::KIND_BIFOCAL  ? bf::attn_tc2_kernel<bf::tc2::KIND_BIFOCAL, false>
+              : kind == bf::tc2::KIND_WINDOW ? bf::attn_tc2_kernel<bf::tc2::KIND_WINDOW, false>
+                                        : bf::attn_tc2_kernel<bf::tc2::KIND_PLAIN, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess) {
     kern<<<static_cast<unsigned>(n_cta), bf::tc2::NTHREADS2, smem, st>>>(ta);
@@ -496,9 +588,15 @@ bf_status_t prefill_impl(bool bifocal_api, const void* q, const void* k, const v
   bf_status_t s = check_params(p, bifocal_api);
   if (s != BF_OK) return s;
   if (!q || !k || !v || !out) return BF_ERR_INVALID;
-  if (!aligned(out, 16)) return BF_ERR_INVALID;
+  if (!aligned(out, 16) || (lse && !aligned(lse, 4))) return BF_ERR_INVALID;
   s = prefill_rope_impl(bifocal_api, q, k, v, dtype, batch, L, p, kcache_out, vcache_out, workspace, ws_bytes, stream);
   if (s != BF_OK) return s;
+  PrefillPlan plan;
+  s = plan_prefill(bifocal_api, dtype, batch, L, p, workspace, ws_bytes, &plan);
+  if (s != BF_OK) return s;
+  if (plan.fused)
+    return fused_attention(plan.kind, q, k, false, v, batch, L, 0, L, plan.G, p, plan.rope, out, lse,
+                           static_cast<cudaStream_t>(stream));
   return prefill_attention_impl(bifocal_api, v, dtype, batch, L, p, out, lse, workspace, ws_bytes, stream);
 }
 
@@ -534,7 +632,8 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
 
   const int D = p->head_dim;
   const int G = bifocal_api ? factor(L, p->w_pretrained) : 1;
-  const bool bif = !window && bifocal_api && (G > 1 || (p->flags & BF_FLAG_FORCE_BIFOCAL)) && p->w0 < L;
+  // BF_FLAG_FORCE_BIFOCAL runs the two-branch kernel whatever G and w0 are, as in prefill
+  const bool bif = !window && bifocal_api && ((p->flags & BF_FLAG_FORCE_BIFOCAL) || (G > 1 && p->w0 < L));
   const int key0 = window ? std::max(0, L - p->w0) : 0;  // a window reads keys L - w0 .. L - 1 only
   const Rope rope = make_rope(p->rope_theta, D, G);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -623,21 +722,60 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
 __device__ __align__(256) uint8_t g_noalloc_scratch[BIFOCAL_NOALLOC_SCRATCH_BYTES];
 
 // Host code cannot use the array's name as a device address: look the address up once per
-// device, with that device current.
+// device, with that device current. The address belongs to the device's current context; a
+// device reset (or a primary context released and created again) gives the module a new
+// address, so the cached one is kept together with the unique id of the context it was read
+// in, and looked up again when the current context is another one.
 constexpr int kMaxDevices = 64;
-void* g_noalloc_ptr[kMaxDevices] = {};
+struct NoallocEntry {
+  void* ptr;
+  unsigned long long ctx_id;
+};
+NoallocEntry g_noalloc[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the current context (0 when it cannot be read: then the address is looked up
+// on every call, which costs a driver call but is always right).
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(a);
+      get_id = reinterpret_cast<CtxGetIdFn>(b);
+    }
+  });
+  if (!get_cur || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 void* noalloc_scratch_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoallocEntry& e = g_noalloc[dev];
+  if (cudaFree(nullptr) != cudaSuccess) return nullptr;  // makes the device's primary context current
+  const unsigned long long id = current_ctx_id();
+  if (!e.ptr || id == 0 || e.ctx_id != id) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_noalloc_ptr[dev] = ptr;
+    e.ptr = ptr;
+    e.ctx_id = id;
   }
-  return g_noalloc_ptr[dev];
+  return e.ptr;
 }
 
 }  // namespace
@@ -759,7 +897,128 @@ bf_status_t decode_paged_impl(const void* q, const void* k_new, const void* v_ne
   return e == cudaSuccess ? BF_OK : BF_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ batched chunks over a paged cache
+bf_status_t chunk_paged_impl(const void* q, const void* k, const void* v, int32_t batch, const int32_t* chunk_lens,
+                             const int32_t* cached_lens, const bf_params_t* p, void* kpool, void* vpool,
+                             int32_t pool_pages, int32_t page_size, const int32_t* block_table, int32_t max_pages,
+                             void* out, float* lse, void* stream) {
+  bf_status_t s = check_params(p, true);
+  if (s != BF_OK) return s;
+  if (!q || !k || !v || !kpool || !vpool || !block_table || !out || !chunk_lens || !cached_lens) return BF_ERR_INVALID;
+  if (batch < 1 || pool_pages < 1 || max_pages < 1) return BF_ERR_INVALID;
+  if (batch > bf::tc2::kMaxSeqs) return BF_ERR_UNSUPPORTED;
+  if (page_size < 16 || page_size % 16 || (128 % page_size && page_size % 128)) return BF_ERR_INVALID;
+  if (static_cast<int64_t>(pool_pages) * page_size > 0x7fffffffLL) return BF_ERR_INVALID;
+  const int D = p->head_dim, g = p->hq / p->hkv;
+  if (D != 128 || p->hq % 2 || g % 2 || (p->flags & BF_FLAG_MMA_SYNC)) return BF_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(kpool, 16) || !aligned(vpool, 16) ||
+      !aligned(out, 16) || !aligned(block_table, 4) || (lse && !aligned(lse, 4)))
+    return BF_ERR_INVALID;
+  const bool window = (p->flags & BF_FLAG_WINDOW) != 0;
+  if (window && p->w0 < 1) return BF_ERR_INVALID;
+  int64_t total = 0;
+  int order[bf::tc2::kMaxSeqs];
+  double work[bf::tc2::kMaxSeqs];
+  for (int i = 0; i < batch; ++i) {
+    const int64_t P0 = cached_lens[i], C = chunk_lens[i];
+    if (P0 < 0 || C < 1 || P0 + C > static_cast<int64_t>(max_pages) * page_size) return BF_ERR_INVALID;
+    total += C;
+    order[i] = i;
+    work[i] = static_cast<double>(C) * (static_cast<double>(P0) + 0.5 * C);  // causal pairs of the chunk
+  }
+  if (total > 0x7fffffffLL) return BF_ERR_INVALID;
+  // launch order: the most work first, so the tail of the grid is light
+  std::sort(order, order + batch, [&](int x, int y) { return work[x] > work[y]; });
+  const int T = static_cast<int>(total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Rope rope = make_rope(p->rope_theta, D, 1);
+
+  // 1. every chunk's keys (original RoPE, bf16) and values into its pages
+  bf::PrepassArgs pa{};
+  pa.q = q;
+  pa.k = k;
+  pa.v = v;
+  pa.batch = 1;
+  pa.L = T;
+  pa.Lk = T;
+  pa.Lc = 0;
+  pa.hq = p->hq;
+  pa.hkv = p->hkv;
+  pa.G = 1;
+  pa.keys_only = 1;
+  pa.kcache = static_cast<bf16*>(kpool);
+  pa.vcache = static_cast<bf16*>(vpool);
+  pa.nseq = batch;
+  pa.block_table = block_table;
+  pa.max_pages = max_pages;
+  pa.page_size = page_size;
+  int row = 0;
+  for (int i = 0; i < batch; ++i) {
+    pa.seq_id[i] = i;
+    pa.seq_P0[i] = cached_lens[i];
+    pa.seq_C[i] = chunk_lens[i];
+    pa.seq_qrow[i] = row;
+    row += chunk_lens[i];
+  }
+  std::memcpy(pa.omega, rope.omega, sizeof(pa.omega));
+  bf::rope_prepass_kernel<bf16, 128><<<static_cast<unsigned>((T + 7) / 8), 256, 0, st>>>(pa);
+  if (cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
+
+  // 2. the fused attention over every sequence's chunk, keys re-phased in the tile loads
+  bf::Tc2Args ta;
+  std::memset(&ta, 0, sizeof(ta));
+  const int seg = std::min(page_size, 128);
+  const int pool_rows = pool_pages * page_size;
+  if (!make_v_map(&ta.qo_map, q, T, p->hq, 1) || !make_v_map(&ta.ko_map, kpool, pool_rows, p->hkv, 1, seg) ||
+      !make_v_map(&ta.v_map, vpool, pool_rows, p->hkv, 1, seg))
+    return BF_ERR_CUDA;
+  ta.out = static_cast<bf16*>(out);
+  ta.lse = lse;
+  ta.hq = p->hq;
+  ta.hkv = p->hkv;
+  ta.batch = 1;
+  ta.w0 = p->w0;
+  ta.scale_log2 = scale_log2(p);
+  ta.src.cache = 1;
+  ta.src.mode = p->mode;
+  ta.src.G = 1;
+  std::memcpy(ta.src.omega, rope.omega, sizeof(ta.src.omega));
+  ta.nseq = batch;
+  ta.total_rows = T;
+  ta.block_table = block_table;
+  ta.max_pages = max_pages;
+  ta.page_size = page_size;
+  ta.seg_rows = seg;
+  int tiles = 0;
+  for (int si = 0; si < batch; ++si) {
+    const int i = order[si];
+    ta.tile_start[si] = tiles;
+    ta.seq_id[si] = i;
+    ta.seq_P0[si] = cached_lens[i];
+    ta.seq_C[si] = chunk_lens[i];
+    ta.seq_G[si] = factor(static_cast<int64_t>(cached_lens[i]) + chunk_lens[i], p->w_pretrained);
+    ta.seq_qrow[si] = pa.seq_qrow[i];
+    tiles += (chunk_lens[i] + bf::tc::BM - 1) / bf::tc::BM;
+  }
+  ta.tile_start[batch] = tiles;
+  const long long n_cta = static_cast<long long>(tiles) * (p->hq / 2);
+  // one kernel kind for the batch: a sequence with G = 1 or w0 >= its length takes the two-branch
+  // kernel as with BF_FLAG_FORCE_BIFOCAL (its long-range forms equal the original ones, or it has
+  // no long-range visit)
+  const int kind = window ? bf::tc2::KIND_WINDOW : bf::tc2::KIND_BIFOCAL;
+  return launch_tc2(kind, true, ta, n_cta, st) == cudaSuccess ? BF_OK : BF_ERR_CUDA;
+}
+
 extern "C" {
+
+bf_status_t bifocal_prefill_chunk_paged(const void* q, const void* k, const void* v, int32_t batch,
+                                        const int32_t* chunk_lens, const int32_t* cached_lens, const bf_params_t* p,
+                                        void* kpool, void* vpool, int32_t pool_pages, int32_t page_size,
+                                        const int32_t* block_table, int32_t max_pages, void* out, float* lse,
+                                        void* stream) {
+  return chunk_paged_impl(q, k, v, batch, chunk_lens, cached_lens, p, kpool, vpool, pool_pages, page_size,
+                          block_table, max_pages, out, lse, stream);
+}
 
 int32_t bifocal_factor(int64_t L, int32_t w_pretrained) {
   if (L < 0 || w_pretrained < 1) return -1;
@@ -794,7 +1053,7 @@ bf_status_t bifocal_decode_paged(const void* q, const void* k_new, const void* v
 
 size_t bifocal_prefill_chunk_workspace_size(int32_t P0, int32_t C, const bf_params_t* p) {
   if (check_params(p, true) != BF_OK || P0 < 0 || C < 1 || static_cast<int64_t>(P0) + C > 0x7fffffff) return 0;
-  return chunk_layout(P0, C, p).total;
+  return chunk_layout(P0, C, p, BF_DTYPE_BF16).total;
 }
 
 bf_status_t bifocal_prefill_chunk(const void* q, const void* k, const void* v, int32_t dtype, int32_t P0, int32_t C,
@@ -871,6 +1130,7 @@ const char* bifocal_status_string(int32_t status) {
     case BF_ERR_TIMEOUT: return "device-side wait timed out";
     case BF_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case BF_ERR_NO_DEVICE: return "no suitable CUDA device";
+    case BF_ERR_RANGE: return "an fp16 QK^T operand was not finite after rounding (|x| >= 65520, inf or NaN)";
     default: return "unknown status";
   }
 }
@@ -882,7 +1142,23 @@ bf_status_t bifocal_last_device_error(void* stream) {
   if (v == 0) return BF_OK;
   const int zero = 0;
   if (cudaMemcpyToSymbol(bf::g_device_status, &zero, sizeof(int)) != cudaSuccess) return BF_ERR_CUDA;
-  return BF_ERR_TIMEOUT;
+  return (v & 0xff) == bf::kDevRange ? BF_ERR_RANGE : BF_ERR_TIMEOUT;
+}
+
+bf_status_t bifocal_test_set_fault(int32_t kind, int32_t arg, int64_t wait_limit_ns) {
+  if (kind < BF_FAULT_NONE || kind > BF_FAULT_DECODE_SKIP_STAGE || wait_limit_ns < 0) return BF_ERR_INVALID;
+  if (kind != BF_FAULT_NONE && arg < 0) return BF_ERR_INVALID;
+  if (cudaDeviceSynchronize() != cudaSuccess) return BF_ERR_CUDA;  // no launch in flight sees a half-set control
+  const int off = -1;
+  const int pre = kind == BF_FAULT_PREFILL_SKIP_FILL ? arg : off;
+  const int dec = kind == BF_FAULT_DECODE_SKIP_STAGE ? arg : off;
+  const unsigned long long lim = wait_limit_ns > 0 ? static_cast<unsigned long long>(wait_limit_ns) : 2000000000ull;
+  if (cudaMemcpyToSymbol(bf::g_skip_fill_prefill, &pre, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(bf::g_skip_stage_decode, &dec, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(bf::g_wait_limit_ns, &lim, sizeof(lim)) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess)
+    return BF_ERR_CUDA;
+  return BF_OK;
 }
 
 int32_t bifocal_device_status_word(void) {

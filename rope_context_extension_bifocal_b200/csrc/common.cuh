@@ -10,15 +10,38 @@
 namespace bf {
 
 // ---------------------------------------------------------------------------------
-// Device status word: bounded waits that give up record a code here and return.
+// Device status word: the first event of a launch sequence that the kernels cannot
+// turn into a correct result records a code here and the kernel carries on or leaves:
+//   kDevTimeout | site << 8   a bounded wait gave up (site numbers the wait in the source)
+//   kDevRange   | site << 8   an operand of the fp16 QK^T product was not finite after
+//                             rounding to fp16 (|x| >= 65520, inf or NaN)
 // Read and cleared by bifocal_last_device_error().
 // ---------------------------------------------------------------------------------
-enum : int { kDevOk = 0, kDevTimeout = 1 };
+enum : int { kDevOk = 0, kDevTimeout = 1, kDevRange = 2 };
 __device__ int g_device_status = 0;
 
-__device__ __forceinline__ void report_timeout(int where) {
-  atomicCAS(&g_device_status, kDevOk, (kDevTimeout | (where << 8)));
+// Wall-clock limit of every bounded wait, in ns (2 s; a test may shorten it through
+// bifocal_test_set_fault so that an expiry costs milliseconds). A wait reads it only once it
+// has already waited kWaitFloorNs (20 ms, far beyond any wait of a healthy launch), so the
+// polling loops of normal operation compare against a constant and never touch global memory.
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
+constexpr unsigned long long kWaitFloorNs = 20000000ull;
+
+// Test-only fault injection, off (-1) unless a test sets it through bifocal_test_set_fault:
+// the producer of CTA 0 skips one whole fill (no expect_tx, no copy), so the wait for it
+// can only expire. Prefill: fill number g_skip_fill_prefill of the K/V ring; decode:
+// stage number g_skip_stage_decode of the split-KV kernel.
+__device__ int g_skip_fill_prefill = -1;
+__device__ int g_skip_stage_decode = -1;
+
+__device__ __forceinline__ void report_status(int code, int where) {
+  if (*reinterpret_cast<volatile int*>(&g_device_status) == kDevOk) atomicCAS(&g_device_status, kDevOk, code | (where << 8));
 }
+__device__ __forceinline__ void report_timeout(int where) { report_status(kDevTimeout, where); }
+
+// fp16 operand range guard: true when rounding x to fp16 gives a finite value (|x| < 65520;
+// from 65520 on round-to-nearest gives inf); false for larger magnitudes, inf and NaN.
+__device__ __forceinline__ bool f16_ok(float x) { return fabsf(x) < 65520.f; }
 
 // ---------------------------------------------------------------------------------
 // RoPE angles. The angle p * omega reaches ~1.3e5 rad at 128K tokens, where an fp32
@@ -74,6 +97,16 @@ __device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
@@ -172,14 +205,17 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
-// Bounded wait: polls the barrier; after ~2 s of wall time it records a timeout and
+// Bounded wait: polls the barrier; after g_wait_limit_ns of wall time it records a timeout and
 // returns false so that the caller can leave instead of hanging the GPU.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, int where) {
   if (mbar_try_wait(bar, phase)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, phase)) return true;
-    if ((it & 63) == 0 && global_ns() - t0 > 2000000000ull) break;
+    if ((it & 63) == 0) {
+      const uint64_t el = global_ns() - t0;
+      if (el > kWaitFloorNs && el > *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns)) break;
+    }
   }
   report_timeout(where);
   return false;
@@ -194,7 +230,8 @@ __device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t phas
     if (mbar_try_wait(bar, phase)) return true;
     if ((it & 63) == 0) {
       if (*abort) return false;
-      if (global_ns() - t0 > 2000000000ull) break;
+      const uint64_t el = global_ns() - t0;
+      if (el > kWaitFloorNs && el > *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns)) break;
     }
   }
   *abort = 1;

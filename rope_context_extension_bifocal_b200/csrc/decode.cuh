@@ -76,8 +76,11 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   uint8_t* sK = smem;                       // [NST][HPC][HALVES][KB][128 B]
   uint8_t* sV = sK + NST * STAGE_KV;        // same
   uint8_t* sCS = sV + NST * STAGE_KV;       // [NST][KB][CS_STRIDE]: correction cos/sin per stage
+  // full[s]: the stage's K/V bytes have landed (producer's expect_tx); tbl[s]: its cos/sin table is
+  // written (one arrive per table-warp lane); empty[s]: every consumer warp is done with the slot
   uint64_t* full = reinterpret_cast<uint64_t*>(sCS + NST * STAGE_CS);
   uint64_t* empty = full + NST;
+  uint64_t* tbl = empty + NST;
   __shared__ int s_abort;  // set when a bounded wait expires: later waits return at once
 
   pdl_launch_dependents();  // the combine may start its prologue; it waits for this grid's writes
@@ -89,7 +92,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   const int bz = paged ? static_cast<int>(blockIdx.z) : 0;
   const int L = paged ? a.seq_lens[bz] : a.L;
   const int G = paged ? (L <= a.w_pretrained ? 1 : (L + a.w_pretrained - 1) / a.w_pretrained) : a.G;
-  const bool bifocal = paged ? ((G > 1 || a.force_bifocal) && a.w0 < L) : (a.bifocal != 0);
+  const bool bifocal = paged ? (a.force_bifocal || (G > 1 && a.w0 < L)) : (a.bifocal != 0);
   const int p = L - 1;
   const int jbeg = a.key0 + blockIdx.x * a.split_len;
   if (jbeg >= L) return;  // a shorter sequence of the batch: no keys in this split (the combine skips it)
@@ -104,7 +107,8 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   if (threadIdx.x == 0) {
     s_abort = 0;
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&full[s], 1 + 32);  // producer's expect_tx + one arrive per producer lane (cos/sin written)
+      mbar_init(&full[s], 1);
+      mbar_init(&tbl[s], 32);
       mbar_init(&empty[s], nconsumers);
     }
     fence_barrier_init();
@@ -117,9 +121,14 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
       prefetch_tensormap(&a.kmap);
       prefetch_tensormap(&a.vmap);
       const uint32_t bytes = 2u * nheads * HALVES * HEAD_TILE;
+      int skip = -1;  // test only: a volatile read inside the branch, so no other CTA waits for the load
+      if ((blockIdx.x | blockIdx.y | blockIdx.z) == 0) skip = *reinterpret_cast<volatile int*>(&g_skip_stage_decode);
+      uint32_t used = 0, par = 0;  // per slot: has a fill been issued, parity of the fills issued
       for (int s = 0; s < nstage; ++s) {
         const int st = s % NST;
         if (s >= NST && !mbar_wait_abortable(&empty[st], ((s / NST) - 1) & 1, 1, &s_abort)) break;
+        if (*reinterpret_cast<volatile int*>(&s_abort)) break;  // a consumer gave up: issue nothing more
+        if (s == skip) continue;
         const int j0 = jbeg + s * KB;
         // Only row p (the new token) comes from the append kernel; every other row was in the
         // cache before this step, so only the stage holding p waits for that grid.
@@ -135,7 +144,14 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
             tma_load_4d(sK + off, &a.kmap, &full[st], 0, hf, head0 + hh, row);
             tma_load_4d(sV + off, &a.vmap, &full[st], 0, hf, head0 + hh, row);
           }
+        used |= 1u << st;
+        par ^= 1u << st;
       }
+      // Every copy issued must have landed before the CTA may exit. The consumers wait for each
+      // stage they read, but after an expired wait they stop waiting, so the producer itself
+      // waits for the last fill of every slot (bounded, not abortable).
+      for (int st = 0; st < NST; ++st)
+        if (used & (1u << st)) mbar_wait(&full[st], ((par >> st) & 1u) ^ 1u, 4);
     }
     return;
   }
@@ -193,7 +209,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
           }
         }
       }
-      mbar_arrive(&full[st]);  // every lane: its table entries are written
+      mbar_arrive(&tbl[st]);  // every lane: its table entries are written
     }
     return;
   }
@@ -235,6 +251,9 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
           xl[e] = x * c - y * sn;
           yl[e] = y * c + x * sn;
         }
+        if (!(f16_ok(xo[0]) & f16_ok(xo[1]) & f16_ok(yo[0]) & f16_ok(yo[1]) & f16_ok(xl[0]) & f16_ok(xl[1]) &
+              f16_ok(yl[0]) & f16_ok(yl[1])))
+          report_status(kDevRange, 42);
         qa_o[kc][sub] = pack_f16x2(xo[0], xo[1]);
         qa_o[kc + KCP][sub] = pack_f16x2(yo[0], yo[1]);
         qa_l[kc][sub] = pack_f16x2(xl[0], xl[1]);
@@ -247,6 +266,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
 #pragma unroll
   for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m_r = -INFINITY, l_r = 0.f;  // softmax state of query row g8 (S layout)
+  bool scores_fin = true;            // every score of a valid key came out finite (fp16 operands in range)
 
   for (int s = 0; s < nstage; ++s) {
     const int st = s % NST;
@@ -255,7 +275,10 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
     const bool tile_long = jt < local_from;
     const bool tile_local = jt + 7 >= local_from;
     // warp-uniform result: the ldmatrix / mma.sync below are warp-collective
-    if (!__all_sync(0xffffffffu, mbar_wait_abortable(&full[st], (s / NST) & 1, 2, &s_abort))) {
+    // the correction table is needed only when the stage holds long-range keys (its phase still
+    // completes for every stage: the table warps arrive on each)
+    if (!__all_sync(0xffffffffu, mbar_wait_abortable(&full[st], (s / NST) & 1, 2, &s_abort) &&
+                                     (j0 >= local_from || mbar_wait_abortable(&tbl[st], (s / NST) & 1, 5, &s_abort)))) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
       continue;
@@ -300,6 +323,10 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
     for (int e = 0; e < 2; ++e) {
       const int j = jt + 2 * t4 + e;
       float x = (j >= local_from) ? so[e] : sl[e];
+      // An fp16 operand that overflowed (|x| >= 65520 rounds to inf) or a NaN key makes the
+      // score inf or NaN (the padding query rows are zero: 0 * inf = NaN), so one test per
+      // score covers every key operand of the stage.
+      if (j < jend) scores_fin &= fabsf(x) < INFINITY;
       x *= a.scale_log2;
       if (j >= jend) x = -INFINITY;
       sc[e] = x;
@@ -355,6 +382,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
     if (lane == 0) mbar_arrive(&empty[st]);
   }
 
+  if (!scores_fin) report_status(kDevRange, 43);
   // partial results of this warp (its own split): rows < g
   l_r += __shfl_xor_sync(0xffffffffu, l_r, 1);
   l_r += __shfl_xor_sync(0xffffffffu, l_r, 2);
@@ -380,7 +408,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
 
 template <int D>
 constexpr int decode_smem_bytes() {
-  return 2 * dec::NST * dec::HPC * (D / 64) * dec::KB * 128 + dec::NST * dec::KB * (D / 2 * 8 + 64) + 2 * dec::NST * 8;
+  return 2 * dec::NST * dec::HPC * (D / 64) * dec::KB * 128 + dec::NST * dec::KB * (D / 2 * 8 + 64) + 3 * dec::NST * 8;
 }
 
 template <int D>

@@ -27,6 +27,7 @@
 #pragma once
 #include "common.cuh"
 #include "prefill_tc.cuh"
+#include "rope_loads.cuh"
 
 namespace bf {
 namespace tc2 {
@@ -36,6 +37,8 @@ constexpr int NSLOT2 = 4;
 constexpr int NTHREADS2 = 384;  // 8 softmax warps, TMA warp, MMA warp, 2 idle warps (register donors)
 constexpr uint32_t Q_BYTES = 32768;  // one Q tile, same layout as a K tile
 constexpr uint32_t COL_SA = 0, COL_SB = 128, COL_OA = 256, COL_OB = 384;
+constexpr int NK3 = 3, NV2 = 2;  // fused form: K ring and V ring
+constexpr int kMaxSeqs = 64;     // sequences of one batched (paged) launch
 
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -109,9 +112,12 @@ __device__ __forceinline__ Schedule make_schedule(int i0, int n_kt, int w0) {
 }  // namespace tc2
 
 struct Tc2Args {
-  CUtensorMap qo_map;  // fp16 [b*hq][L][128], box (64, 128, 1), 128B swizzle
+  // FUSED = false: the RoPE pass's fp16 operand forms, [b*h][L][128], box (64, 128, 1).
+  // FUSED = true: qo_map is the raw bf16 q [b][Lq][hq][128] and ko_map the raw bf16 keys
+  // [b][L][hkv][128] (or the cache of original-RoPE keys), box (64, 1, 128, 1); ql/kl unused.
+  CUtensorMap qo_map;
   CUtensorMap ql_map;
-  CUtensorMap ko_map;  // fp16 [b*hkv][L][128]
+  CUtensorMap ko_map;
   CUtensorMap kl_map;
   CUtensorMap v_map;   // bf16 [b][L][hkv][128], box (64, 1, 128, 1)
   __nv_bfloat16* out;  // [b, Lq, hq, 128]
@@ -121,27 +127,78 @@ struct Tc2Args {
   // q_off = 0 and Lq = L; a chunk over a cache has q_off = the cached length); keys 0 .. L-1
   int q_off, Lq;
   float scale_log2;
+  RopeSrc src;  // angles of the fused loads (FUSED only)
+  // A batch of chunks over a paged cache (FUSED only, nseq > 0). Launch-order entry s is the
+  // chunk of sequence seq_id[s] (its block-table row): cached length seq_P0[s], chunk length
+  // seq_C[s], factor seq_G[s], first row seq_qrow[s] of the packed q / out / lse rows (total_rows
+  // in all); query tiles tile_start[s] .. tile_start[s + 1] - 1 of the grid are its. Key j of
+  // that sequence is pool row block_table[seq_id[s] * max_pages + j / page_size] * page_size +
+  // j % page_size, and K / V tiles arrive in segments of seg_rows = min(page_size, 128) rows.
+  int nseq, total_rows;
+  const int* block_table;
+  int max_pages, page_size, seg_rows;
+  int tile_start[tc2::kMaxSeqs + 1];
+  int seq_id[tc2::kMaxSeqs], seq_P0[tc2::kMaxSeqs], seq_C[tc2::kMaxSeqs], seq_G[tc2::kMaxSeqs],
+      seq_qrow[tc2::kMaxSeqs];
 };
 
-template <int KIND>
+// FUSED = false: Q and K tiles come by TMA from the RoPE pass's fp16 forms; K and V share a
+// ring of four slots (fill n in slot n % 4: K of visit v is fill 2v, V fill 2v + 1).
+// FUSED = true: TMA brings the raw bf16 tiles; warps 10 and 11 rotate Q and K in place into
+// fp16 operands (rope_loads.cuh); K has its own ring of three slots, V of two. No rotated
+// copy of q or k exists in HBM.
+template <int KIND, bool FUSED>
 __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __grid_constant__ Tc2Args a) {
   using namespace tc2;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ uint64_t full[NSLOT2], empty[NSLOT2], s_full[2], p_ready[2], o_done[2], q_full, q_free, mma_drain;
+  // fused rings: K raw landed / K operand ready / K slot free; V landed / V slot free; raw Q landed
+  __shared__ uint64_t kraw[NK3], kfull[NK3], kempty[NK3], vfull[NV2], vempty[NV2], q_raw, v_fix[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_qt = (a.Lq + BM - 1) / BM;
   const int pairs = a.hq / 2;
-  const int per_tile = pairs * a.batch;
-  const int qt = n_qt - 1 - static_cast<int>(blockIdx.x) / per_tile;  // heaviest first
-  const int rem = static_cast<int>(blockIdx.x) % per_tile;
-  const int hp = rem % pairs, b = rem / pairs;
+  // This CTA's query tile: rows q_off + qt*BM .. of a sequence with Lq query rows after q_off
+  // cached ones (L = q_off + Lq keys), factor G; b is its batch index (dense) or block-table
+  // row (paged); qrow0 its first row in out / lse.
+  int qt, hp, b, q_off, Lq, L, G, qrow0;
+  const bool paged = FUSED && a.nseq > 0;
+  if (paged) {
+    const int tile = static_cast<int>(blockIdx.x) / pairs;
+    hp = static_cast<int>(blockIdx.x) % pairs;
+    int sq = 0;
+    while (sq + 1 < a.nseq && a.tile_start[sq + 1] <= tile) ++sq;
+    b = a.seq_id[sq];
+    q_off = a.seq_P0[sq];
+    Lq = a.seq_C[sq];
+    G = a.seq_G[sq];
+    qrow0 = a.seq_qrow[sq];
+    qt = (Lq + BM - 1) / BM - 1 - (tile - a.tile_start[sq]);  // heaviest first within the sequence
+  } else {
+    // kv-head major: the CTAs resident at one time share one kv head's K and V tiles (the key
+    // forms of one head fit in L2 at 128K, those of all eight do not: with the query tiles of
+    // every head in flight, K and V were read from DRAM ~23 times over), heaviest query tile
+    // first within a head
+    const int n_qt = (a.Lq + BM - 1) / BM;
+    const int ppk = pairs / a.hkv;  // head pairs per kv head
+    const int idx = static_cast<int>(blockIdx.x);
+    const int pk = idx % ppk;
+    const int rest = idx / ppk;
+    qt = n_qt - 1 - rest % n_qt;
+    const int bk = rest / n_qt;  // batch * hkv + kv head
+    b = bk / a.hkv;
+    hp = (bk % a.hkv) * ppk + pk;
+    q_off = a.q_off;
+    Lq = a.Lq;
+    G = a.src.G;
+    qrow0 = b * a.Lq;
+  }
+  L = q_off + Lq;
   const int h0 = 2 * hp;  // heads h0 (tile A) and h0 + 1 (tile B), same kv head
   const int kvh = h0 / (a.hq / a.hkv);
-  const int i0 = a.q_off + qt * BM;  // absolute position of the tile's first query row
-  const int n_kt = (min(i0 + BM, a.q_off + a.Lq) + BN - 1) / BN;
+  const int i0 = q_off + qt * BM;  // absolute position of the tile's first query row
+  const int n_kt = (min(i0 + BM, L) + BN - 1) / BN;
   const Schedule sch = make_schedule<KIND>(i0, n_kt, a.w0);
   const int nv = sch.total();
   const bool has_long = sch.n_long() > 0;
@@ -149,7 +206,8 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
   const bool reload_q = has_long && has_orig;
   const int v_sw = sch.n_long();  // first local visit (when reload_q)
   const uint32_t qbase = smem_u32(smem);                  // Q_A, Q_B
-  const uint32_t slots = qbase + 2 * Q_BYTES;             // K/V ring
+  const uint32_t slots = qbase + 2 * Q_BYTES;             // K/V ring; fused: K slots, then V slots
+  const uint32_t vslots = slots + (FUSED ? NK3 : 0) * SLOT_BYTES;
 
   if (threadIdx.x == 0) {
     s_abort = 0;
@@ -157,12 +215,24 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
+    for (int i = 0; i < NK3; ++i) {
+      mbar_init(&kraw[i], 1);
+      mbar_init(&kfull[i], rl::NXF);
+      mbar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < NV2; ++i) {
+      mbar_init(&vfull[i], 1);
+      mbar_init(&vempty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_ready[i], 4);
       mbar_init(&o_done[i], 1);
     }
-    mbar_init(&q_full, 1);
+    mbar_init(&q_raw, 1);
+    mbar_init(&v_fix[0], rl::NXF);  // one per visit of a tile past a paged sequence's end (at most two:
+    mbar_init(&v_fix[1], rl::NXF);  // its long-range half and its local half), each used once
+    mbar_init(&q_full, FUSED ? rl::NXF : 1);
     mbar_init(&q_free, 1);
     mbar_init(&mma_drain, 1);
     fence_barrier_init();
@@ -177,90 +247,234 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
   fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  // Registers: launched at 168 per thread (384 threads). Warpgroup 2 (TMA, MMA, two idle
-  // warps) gives 72 of them back and the two softmax warpgroups take 32 more each:
+  // Barriers and slots of visit v's K and V tiles, for either ring layout.
+  auto k_full = [&](int v) -> uint64_t* { return FUSED ? &kfull[v % NK3] : &full[(2 * v) % NSLOT2]; };
+  auto k_full_ph = [&](int v) -> uint32_t { return FUSED ? (v / NK3) & 1 : ((2 * v) / NSLOT2) & 1; };
+  auto k_empty = [&](int v) -> uint64_t* { return FUSED ? &kempty[v % NK3] : &empty[(2 * v) % NSLOT2]; };
+  auto k_slot = [&](int v) -> int { return FUSED ? v % NK3 : (2 * v) % NSLOT2; };
+  auto v_full = [&](int v) -> uint64_t* { return FUSED ? &vfull[v % NV2] : &full[(2 * v + 1) % NSLOT2]; };
+  auto v_full_ph = [&](int v) -> uint32_t { return FUSED ? (v / NV2) & 1 : ((2 * v + 1) / NSLOT2) & 1; };
+  auto v_empty = [&](int v) -> uint64_t* { return FUSED ? &vempty[v % NV2] : &empty[(2 * v + 1) % NSLOT2]; };
+  auto v_slot = [&](int v) -> int { return FUSED ? v % NV2 : (2 * v + 1) % NSLOT2; };
+
+  // Registers: launched at 168 per thread (384 threads). Warpgroup 2 (TMA, MMA, two idle or
+  // transform warps) gives 72 of them back and the two softmax warpgroups take 32 more each:
   // 2 * 128 * 200 + 128 * 96 = 63488 <= 384 * 168, so the increase never waits for registers
   // that the block does not hold. Each role branch starts with its own setmaxnreg so that the
   // compiler allocates each branch within its own limit.
   if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 96;");
+    // the fused form's transform warps take the 8 registers left over: 2 * 128 * 200 + 128 * 104
+    // = 384 * 168 exactly
+    if (FUSED)
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 104;");
+    else
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 96;");
     if (warp == 8) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
         prefetch_tensormap(&a.qo_map);
         prefetch_tensormap(&a.ko_map);
         prefetch_tensormap(&a.v_map);
-        if (KIND == KIND_BIFOCAL) {
+        if (KIND == KIND_BIFOCAL && !FUSED) {
           prefetch_tensormap(&a.ql_map);
           prefetch_tensormap(&a.kl_map);
         }
-        const int qrow = b * a.hq + h0;
-        auto load_q = [&](const CUtensorMap* m) {
-          mbar_arrive_expect_tx(&q_full, 2 * Q_BYTES);
+        int skip = -1;  // test only: never issue this fill (a volatile read inside the branch)
+        if (blockIdx.x == 0) skip = *reinterpret_cast<volatile int*>(&g_skip_fill_prefill);
+        uint32_t used = 0, par = 0;    // unfused ring: per slot, has a fill been issued, parity of the fills
+        uint32_t kused = 0, kpar = 0;  // fused K ring (raw landed barriers)
+        uint32_t vused = 0, vpar = 0;  // fused V ring
+        // Q: both heads; fused: raw rows of this call (map over Lq rows), else the rotated form
+        auto load_q = [&](bool lng) {
+          uint64_t* bar = FUSED ? &q_raw : &q_full;
+          mbar_arrive_expect_tx(bar, 2 * Q_BYTES);
           for (int x = 0; x < 2; ++x) {
             uint8_t* dst = smem + x * Q_BYTES;
-            tma_load_3d(dst, m, &q_full, 0, qt * BM, qrow + x);
-            tma_load_3d(dst + HALF_BYTES, m, &q_full, 64, qt * BM, qrow + x);
+            if (FUSED) {
+              // raw rows [b][Lq][hq][128], or the packed rows of a paged batch [1][total_rows][hq][128]
+              const int row = (paged ? qrow0 : 0) + qt * BM, bb = paged ? 0 : b;
+              tma_load_4d(dst, &a.qo_map, bar, 0, h0 + x, row, bb);
+              tma_load_4d(dst + HALF_BYTES, &a.qo_map, bar, 64, h0 + x, row, bb);
+            } else {
+              const CUtensorMap* m = lng ? &a.ql_map : &a.qo_map;
+              tma_load_3d(dst, m, bar, 0, qt * BM, b * a.hq + h0 + x);
+              tma_load_3d(dst + HALF_BYTES, m, bar, 64, qt * BM, b * a.hq + h0 + x);
+            }
           }
         };
-        load_q(has_long ? &a.ql_map : &a.qo_map);
+        load_q(has_long);
+        int q_loads = 1;
         const int krow = b * a.hkv + kvh;
-        int n = 0;
-        bool ok = true;
-        for (int v = 0; v < nv && ok; ++v) {
-          if (reload_q && v == v_sw) {
-            // every QK^T with the long-range Q has finished reading it
-            if (!mbar_wait_abortable(&q_free, 0, 12, &s_abort)) {
-              ok = false;
-              break;
-            }
-            load_q(&a.qo_map);
-          }
+        // One fill: the K (x = 0) or V (x = 1) tile of visit v, fill number 2v + x, into its slot
+        // once the slot's previous tile is consumed. False when a wait gave up.
+        auto fill = [&](int x, int v) -> bool {
+          const int n = 2 * v + x;
+          const int use = FUSED ? (x == 0 ? v / NK3 : v / NV2) : n / NSLOT2;
+          uint64_t* freed = x == 0 ? k_empty(v) : v_empty(v);
+          if (use > 0 && !mbar_wait_abortable(freed, (use - 1) & 1, 10, &s_abort)) return false;
+          if (n == skip) return true;
           int t, kind;
           sch.visit(v, t, kind);
           const bool lng = kind == LONG_FULL || kind == LONG_ONLY;
-          for (int x = 0; x < 2; ++x, ++n) {
-            const int slot = n % NSLOT2, use = n / NSLOT2;
-            if (use > 0 && !mbar_wait_abortable(&empty[slot], (use - 1) & 1, 10, &s_abort)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&full[slot], SLOT_BYTES);
-            uint8_t* dst = smem + 2 * Q_BYTES + slot * SLOT_BYTES;
+          const int sl = x == 0 ? k_slot(v) : v_slot(v);
+          if (FUSED) {
             if (x == 0) {
-              const CUtensorMap* m = lng ? &a.kl_map : &a.ko_map;
-              tma_load_3d(dst, m, &full[slot], 0, t * BN, krow);
-              tma_load_3d(dst + HALF_BYTES, m, &full[slot], 64, t * BN, krow);
+              kused |= 1u << sl;
+              kpar ^= 1u << sl;
             } else {
-              tma_load_4d(dst, &a.v_map, &full[slot], 0, kvh, t * BN, b);
-              tma_load_4d(dst + HALF_BYTES, &a.v_map, &full[slot], 64, kvh, t * BN, b);
+              vused |= 1u << sl;
+              vpar ^= 1u << sl;
+            }
+          } else {
+            used |= 1u << sl;
+            par ^= 1u << sl;
+          }
+          uint64_t* bar = FUSED ? (x == 0 ? &kraw[sl] : &vfull[sl]) : &full[sl];
+          uint8_t* dst = smem + ((x == 0 ? slots : vslots) - qbase) + sl * SLOT_BYTES;
+          if (paged) {
+            // segments of seg_rows keys, each one page's rows of the pool; segments wholly past
+            // the sequence's end are not loaded (their K rows are zeroed by the transform, their
+            // V rows by the fix-up of each visit of that tile)
+            const CUtensorMap* m = x == 0 ? &a.ko_map : &a.v_map;
+            const int nseg = BN / a.seg_rows;
+            const int nvalid = min(nseg, (L - t * BN + a.seg_rows - 1) / a.seg_rows);
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nvalid * a.seg_rows) * 256u);
+            for (int sg = 0; sg < nvalid; ++sg) {
+              const int j = t * BN + sg * a.seg_rows;
+              const int row =
+                  a.block_table[static_cast<long long>(b) * a.max_pages + j / a.page_size] * a.page_size +
+                  j % a.page_size;
+              uint8_t* d0 = dst + sg * a.seg_rows * 128;
+              tma_load_4d(d0, m, bar, 0, kvh, row, 0);
+              tma_load_4d(d0 + HALF_BYTES, m, bar, 64, kvh, row, 0);
+            }
+            return true;
+          }
+          mbar_arrive_expect_tx(bar, SLOT_BYTES);
+          if (x == 1 || FUSED) {
+            const CUtensorMap* m = x == 0 ? &a.ko_map : &a.v_map;
+            tma_load_4d(dst, m, bar, 0, kvh, t * BN, b);
+            tma_load_4d(dst + HALF_BYTES, m, bar, 64, kvh, t * BN, b);
+          } else {
+            const CUtensorMap* m = lng ? &a.kl_map : &a.ko_map;
+            tma_load_3d(dst, m, bar, 0, t * BN, krow);
+            tma_load_3d(dst + HALF_BYTES, m, bar, 64, t * BN, krow);
+          }
+          return true;
+        };
+        if (FUSED) {
+          // K runs two visits ahead of V (step u: K(u), then V(u - 2)), so no K fill waits behind
+          // a V slot: a raw K tile still has to be rotated after it lands. The raw Q reload goes
+          // out as soon as q_free has completed: tried at step v_sw, waited for at step v_sw + 1,
+          // after V(v_sw - 1), the last fill the MMA needs before it can reach q_free.
+          bool q_pending = reload_q;
+          for (int u = 0; u < nv + 2; ++u) {
+            if (u < nv && !fill(0, u)) break;
+            if (u >= 2 && u - 2 < nv && !fill(1, u - 2)) break;
+            if (q_pending && u >= v_sw) {
+              if (u > v_sw || mbar_try_wait(&q_free, 0)) {
+                if (!mbar_wait_abortable(&q_free, 0, 12, &s_abort)) break;
+                load_q(false);
+                ++q_loads;
+                q_pending = false;
+              }
             }
           }
+        } else {
+          for (int v = 0; v < nv; ++v) {
+            if (reload_q && v == v_sw) {
+              // every QK^T with the long-range Q has finished reading it
+              if (!mbar_wait_abortable(&q_free, 0, 12, &s_abort)) break;
+              load_q(false);
+              ++q_loads;
+            }
+            if (!fill(0, v) || !fill(1, v)) break;
+          }
         }
-        // drain: every fill issued must have landed before the CTA may exit
-        const int first = n > NSLOT2 ? n - NSLOT2 : 0;
-        for (int k = first; k < n; ++k) mbar_wait(&full[k % NSLOT2], (k / NSLOT2) & 1, 11);
-        mbar_wait(&q_full, reload_q ? 1 : 0, 13);
+        // drain: every copy issued must have landed before the CTA may exit: the last fill of
+        // every slot (the ones before it were consumed, or a later fill could not have been
+        // issued) and the last Q load
+        if (FUSED) {
+          for (int sl = 0; sl < NK3; ++sl)
+            if (kused & (1u << sl)) mbar_wait(&kraw[sl], ((kpar >> sl) & 1u) ^ 1u, 11);
+          for (int sl = 0; sl < NV2; ++sl)
+            if (vused & (1u << sl)) mbar_wait(&vfull[sl], ((vpar >> sl) & 1u) ^ 1u, 11);
+          mbar_wait(&q_raw, (q_loads - 1) & 1, 13);
+        } else {
+          for (int sl = 0; sl < NSLOT2; ++sl)
+            if (used & (1u << sl)) mbar_wait(&full[sl], ((par >> sl) & 1u) ^ 1u, 11);
+          mbar_wait(&q_full, (q_loads - 1) & 1, 13);
+        }
+      }
+    } else if (FUSED && warp >= 10) {
+      // ------------------------------------------------------------ fused RoPE: rotate tiles in place
+      const int pt = (warp - 10) * 32 + lane;
+      const int cch = pt & 7, r0 = pt >> 3;
+      // Q: raw rows landed -> the first form (long-range when the tile has long visits)
+      if (warp_wait(&q_raw, 0, 14, &s_abort)) {
+        rope_query_tiles(qbase, a.src, G, has_long ? rl::FORM_LONG : rl::FORM_ORIG, i0, cch, r0);
+        fence_proxy_async_smem();
+        mbar_arrive(&q_full);
+        Rot8 st, s8;
+        int cur_form = -1, next_t = -1, run = 0;
+        int n_fixed = 0;  // visits of a tile past a paged sequence's end handled so far
+        for (int v = 0; v < nv; ++v) {
+          int t, kind;
+          sch.visit(v, t, kind);
+          const int form = (kind == LONG_FULL || kind == LONG_ONLY) ? rl::FORM_LONG : rl::FORM_ORIG;
+          const int sl = v % NK3;
+          if (!warp_wait(&kraw[sl], (v / NK3) & 1, 16, &s_abort)) break;
+          const bool linear = form_linear(a.src, G, form);
+          if (linear && !(a.src.cache && form == rl::FORM_ORIG)) {
+            if (form != cur_form) rot_step(s8, a.src, G, form, true, 8, 8 * cch);
+            if (form != cur_form || t != next_t || run >= rl::ANCHOR_EVERY) {
+              rot_exact(st, a.src, G, form, true, static_cast<long long>(t) * BN + r0, 8 * cch);
+              run = 0;
+            }
+            cur_form = form;
+            next_t = t + 1;
+            ++run;
+          } else {
+            cur_form = -1;  // st is not kept (exact angles per row, or no rotation): anchor the next run
+          }
+          rope_key_tile(slots + sl * SLOT_BYTES, a.src, G, form, linear, t * BN, L, cch, r0, st, s8);
+          fence_proxy_async_smem();
+          mbar_arrive(&kfull[sl]);
+          if (paged && t * BN + BN > L && n_fixed < 2) {
+            // this tile runs past the sequence's end (it may be visited twice, once per branch):
+            // its V rows there hold whatever the pool holds; zero them once the tile has landed
+            // (the MMA waits for v_fix before this visit's PV)
+            if (!warp_wait(&vfull[v % NV2], (v / NV2) & 1, 18, &s_abort)) break;
+            zero_tile_rows(vslots + (v % NV2) * SLOT_BYTES, L - t * BN, cch, r0);
+            fence_proxy_async_smem();
+            mbar_arrive(&v_fix[n_fixed++]);
+          }
+          if (reload_q && v == v_sw) {
+            // the first original-form visit's K is ready; now the original-form Q: the producer
+            // reloads the raw rows once every long-range QK^T has read the first form
+            if (!warp_wait(&q_raw, 1, 15, &s_abort)) break;
+            rope_query_tiles(qbase, a.src, G, rl::FORM_ORIG, i0, cch, r0);
+            fence_proxy_async_smem();
+            mbar_arrive(&q_full);
+          }
+        }
       }
     } else if (warp == 9) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0 && nv > 0) {
+        int n_fix = 0;  // visits of a tile past the sequence's end seen so far (paged: V tail zeroed)
         bool ok = mbar_wait_abortable(&q_full, 0, 20, &s_abort);
         fence_after();
-        auto kslot = [&](int v) { return (2 * v) % NSLOT2; };
-        auto vslot = [&](int v) { return (2 * v + 1) % NSLOT2; };
-        auto kphase = [&](int v) { return static_cast<uint32_t>(((2 * v) / NSLOT2) & 1); };
-        auto vphase = [&](int v) { return static_cast<uint32_t>(((2 * v + 1) / NSLOT2) & 1); };
         // The issuing thread waits on each tcgen05.mma before it can issue the next one, so any
         // arithmetic between two MMAs of a group adds to the group's time (it halved the tensor
         // rate here). Descriptors are therefore formed once, and the eight K-steps of a group
         // only add constants to the start-address field (addresses stay below 2^18, so the
         // field never carries into the next one).
         const uint64_t dqa = k_desc(qbase, 0), dqb = k_desc(qbase + Q_BYTES, 0);
-        const uint64_t dk0 = k_desc(slots, 0), dv0 = v_desc(slots, 0);
+        const uint64_t dk0 = k_desc(slots, 0), dv0 = v_desc(vslots, 0);
         auto qk = [&](int x, int v) {
           const uint64_t a0 = x == 0 ? dqa : dqb;
-          const uint64_t b0 = dk0 + static_cast<uint64_t>(kslot(v) * (SLOT_BYTES >> 4));
+          const uint64_t b0 = dk0 + static_cast<uint64_t>(k_slot(v) * (SLOT_BYTES >> 4));
           const uint32_t d = tmem + (x == 0 ? COL_SA : COL_SB);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
@@ -270,7 +484,7 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
           mma_commit(&s_full[x]);
         };
         auto pv = [&](int x, int v) {
-          const uint64_t b0 = dv0 + static_cast<uint64_t>(vslot(v) * (SLOT_BYTES >> 4));
+          const uint64_t b0 = dv0 + static_cast<uint64_t>(v_slot(v) * (SLOT_BYTES >> 4));
           const uint32_t p_col = tmem + (x == 0 ? COL_SA : COL_SB);
           const uint32_t o_col = tmem + (x == 0 ? COL_OA : COL_OB);
           const uint32_t acc0 = v > 0;
@@ -280,20 +494,28 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
           mma_commit(&o_done[x]);
         };
         // visit 0: S_A, S_B
-        if (ok) ok = mbar_wait_abortable(&full[kslot(0)], kphase(0), 21, &s_abort);
+        if (ok) ok = mbar_wait_abortable(k_full(0), k_full_ph(0), 21, &s_abort);
         if (ok) {
           fence_after();
           qk(0, 0);
           qk(1, 0);
-          mma_commit(&empty[kslot(0)]);
+          mma_commit(k_empty(0));
           if (reload_q && v_sw == 1) mma_commit(&q_free);
         }
         for (int v = 0; v < nv && ok; ++v) {
           // O_A += P_A(v) V(v)
           if (!mbar_wait_abortable(&p_ready[0], v & 1, 22, &s_abort) ||
-              !mbar_wait_abortable(&full[vslot(v)], vphase(v), 23, &s_abort)) {
+              !mbar_wait_abortable(v_full(v), v_full_ph(v), 23, &s_abort)) {
             ok = false;
             break;
+          }
+          if (paged) {
+            int tv, kv;
+            sch.visit(v, tv, kv);
+            if (tv * BN + BN > L && n_fix < 2 && !mbar_wait_abortable(&v_fix[n_fix++], 0, 28, &s_abort)) {
+              ok = false;
+              break;
+            }
           }
           fence_after();
           pv(0, v);
@@ -303,7 +525,7 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
               ok = false;
               break;
             }
-            if (!mbar_wait_abortable(&full[kslot(v + 1)], kphase(v + 1), 25, &s_abort)) {
+            if (!mbar_wait_abortable(k_full(v + 1), k_full_ph(v + 1), 25, &s_abort)) {
               ok = false;
               break;
             }
@@ -317,10 +539,10 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
           }
           fence_after();
           pv(1, v);
-          mma_commit(&empty[vslot(v)]);
+          mma_commit(v_empty(v));
           if (more) {
             qk(1, v + 1);
-            mma_commit(&empty[kslot(v + 1)]);
+            mma_commit(k_empty(v + 1));
             if (reload_q && v + 2 == v_sw) mma_commit(&q_free);
           }
         }
@@ -484,14 +706,14 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
     if (ok && nv > 0 && __all_sync(0xffffffffu, mbar_wait_abortable(&o_done[x], (nv - 1) & 1, 32, &s_abort))) {
       fence_after();
       const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      const int rel = i - a.q_off;  // row of this query in out / lse
-      __nv_bfloat16* orow = a.out + ((static_cast<long long>(b) * a.Lq + rel) * a.hq + h) * D;
+      const int rel = i - q_off;  // row of this query in the call's rows
+      __nv_bfloat16* orow = a.out + ((static_cast<long long>(qrow0) + rel) * a.hq + h) * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < 128; c0 += 32) {
         float ov[32];
         tmem_ld32(o_col + c0, ov);
         wait_ld();
-        if (rel < a.Lq) {
+        if (rel < Lq) {
 #pragma unroll
           for (int u = 0; u < 32; u += 8) {
             uint4 w;
@@ -503,8 +725,16 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
           }
         }
       }
-      if (a.lse && rel < a.Lq)
-        a.lse[(static_cast<long long>(b) * a.hq + h) * a.Lq + rel] = (m_ref + __log2f(l_sum)) * 0.69314718055994530942f;
+      // Every valid row has at least one key in range, so its normaliser is finite and positive
+      // unless an fp16 operand overflowed (an inf score makes the row NaN): report it.
+      if (rel < Lq && !(l_sum > 0.f && l_sum < INFINITY && m_ref > -INFINITY && m_ref < INFINITY))
+        report_status(kDevRange, 45);
+      if (a.lse && rel < Lq) {
+        // dense: [b, hq, Lq]; a paged batch: [hq, total_rows] over the packed rows
+        const long long li = paged ? static_cast<long long>(h) * a.total_rows + qrow0 + rel
+                                   : (static_cast<long long>(b) * a.hq + h) * a.Lq + rel;
+        a.lse[li] = (m_ref + __log2f(l_sum)) * 0.69314718055994530942f;
+      }
     }
   }
 
@@ -514,6 +744,8 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
   if (warp == 9) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NCOLS));
 }
 
-constexpr int attn_tc2_smem_bytes() { return 2 * tc2::Q_BYTES + tc2::NSLOT2 * tc::SLOT_BYTES; }
+constexpr int attn_tc2_smem_bytes(bool fused = false) {
+  return 2 * tc2::Q_BYTES + (fused ? tc2::NK3 + tc2::NV2 : tc2::NSLOT2) * tc::SLOT_BYTES;
+}
 
 }  // namespace bf

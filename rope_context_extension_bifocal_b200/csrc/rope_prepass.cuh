@@ -40,6 +40,7 @@ struct PrepassArgs {
   int G;
   int mode;       // 0 = frequency interpolation, 1 = position aliasing
   int need_long;  // write Ql / Kl
+  int keys_only;  // skip q: only the cache rows (kcache / vcache) and the key forms that are non-null
   __half* Qo;
   __half* Ql;
   __half* Ko;
@@ -54,6 +55,15 @@ struct PrepassArgs {
   const void* q_norm_w;
   const void* k_norm_w;
   float norm_eps;
+  // A batch of chunks appended to a paged cache (keys_only, nseq > 0; batch 1, L = the packed
+  // rows): packed row g belongs to entry s with seq_qrow[s] <= g < seq_qrow[s] + seq_C[s], at
+  // position seq_P0[s] + g - seq_qrow[s] of the sequence whose block-table row is seq_id[s];
+  // position p of it is cache row block_table[seq_id[s] * max_pages + p / page_size] *
+  // page_size + p % page_size.
+  int nseq;
+  const int* block_table;
+  int max_pages, page_size;
+  int seq_id[64], seq_P0[64], seq_C[64], seq_qrow[64];
 };
 
 template <typename T>
@@ -112,7 +122,15 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
   if (gpos >= static_cast<long long>(a.batch) * a.L) return;
   const int b = static_cast<int>(gpos / a.L);
   const int r_in = static_cast<int>(gpos % a.L);  // row of the input
-  const int p = a.pos0 + r_in;                     // absolute position
+  int p = a.pos0 + r_in;                           // absolute position
+  long long crow = static_cast<long long>(b) * a.Lc + p;  // row of kcache / vcache
+  if (a.nseq > 0) {
+    int sq = 0;
+    while (sq + 1 < a.nseq && a.seq_qrow[sq + 1] <= r_in) ++sq;
+    p = a.seq_P0[sq] + (r_in - a.seq_qrow[sq]);
+    crow = static_cast<long long>(a.block_table[static_cast<long long>(a.seq_id[sq]) * a.max_pages + p / a.page_size]) *
+               a.page_size + p % a.page_size;
+  }
   const int grp = lane >> 3, l8 = lane & 7;
   if (l8 >= LANES_PER_ROW) return;
   const int k0 = l8 * NPAIR;  // first pair index this lane owns
@@ -137,7 +155,7 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
   const Tin* kb = static_cast<const Tin*>(a.k);
   const Tin* vb = static_cast<const Tin*>(a.v);
   const int rows = a.hq + a.hkv;
-  for (int r = grp; r < rows; r += 4) {
+  for (int r = (a.keys_only ? a.hq : 0) + grp; r < rows; r += 4) {
     const bool is_q = r < a.hq;
     const int h = is_q ? r : r - a.hq;
     const int H = is_q ? a.hq : a.hkv;
@@ -180,19 +198,28 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
       yl1[i] = u * cl[i] - w * sl[i];
       yl2[i] = w * cl[i] + u * sl[i];
     }
+    // fp16 range guard on the QK^T operands (a larger magnitude would round to inf)
+    bool fin = true;
+#pragma unroll
+    for (int i = 0; i < NPAIR; ++i) {
+      fin &= f16_ok(yo1[i]) & f16_ok(yo2[i]);
+      if (a.need_long) fin &= f16_ok(yl1[i]) & f16_ok(yl2[i]);
+    }
+    if (!fin) report_status(kDevRange, 40);
     // head-major rows: Q has the input's L rows, K the Lk rows of keys 0 .. Lk-1
     const long long hm = is_q ? ((static_cast<long long>(b) * H + h) * a.L + r_in) * D
                               : ((static_cast<long long>(b) * H + h) * a.Lk + p) * D;
-    __half* dst_o = (is_q ? a.Qo : a.Ko) + hm;
-    store8_f16(dst_o + k0, yo1);
-    store8_f16(dst_o + P + k0, yo2);
+    if (__half* dst_o = is_q ? a.Qo : a.Ko) {
+      store8_f16(dst_o + hm + k0, yo1);
+      store8_f16(dst_o + hm + P + k0, yo2);
+    }
     if (a.need_long) {
       __half* dst_l = (is_q ? a.Ql : a.Kl) + hm;
       store8_f16(dst_l + k0, yl1);
       store8_f16(dst_l + P + k0, yl2);
     }
     if (!is_q && a.kcache) {
-      __nv_bfloat16* dc = a.kcache + ((static_cast<long long>(b) * a.Lc + p) * a.hkv + h) * D;
+      __nv_bfloat16* dc = a.kcache + (crow * a.hkv + h) * D;
       store8_bf16(dc + k0, yo1);
       store8_bf16(dc + P + k0, yo2);
     }
@@ -201,7 +228,7 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
   if (a.Vb || a.vcache) {
     for (int h = grp; h < a.hkv; h += 4) {
       const long long off = ((static_cast<long long>(b) * a.L + r_in) * a.hkv + h) * D;
-      const long long coff = ((static_cast<long long>(b) * a.Lc + p) * a.hkv + h) * D;
+      const long long coff = (crow * a.hkv + h) * D;
       Vec8<Tin> x1, x2;
       x1.load(vb + off + k0);
       x2.load(vb + off + P + k0);
@@ -266,6 +293,9 @@ __global__ void __launch_bounds__(256) cache_rephase_kernel(const __grid_constan
       u[i] = x1.get(i);
       w[i] = x2.get(i);
     }
+    bool fin = true;
+#pragma unroll
+    for (int i = 0; i < NPAIR; ++i) fin &= f16_ok(u[i]) & f16_ok(w[i]);
     __half* dst_o = a.Ko + (static_cast<long long>(h) * a.Lk + j) * D;
     store8_f16(dst_o + k0, u);
     store8_f16(dst_o + P + k0, w);
@@ -276,10 +306,13 @@ __global__ void __launch_bounds__(256) cache_rephase_kernel(const __grid_constan
         y1[i] = u[i] * cc[i] - w[i] * sc[i];
         y2[i] = w[i] * cc[i] + u[i] * sc[i];
       }
+#pragma unroll
+      for (int i = 0; i < NPAIR; ++i) fin &= f16_ok(y1[i]) & f16_ok(y2[i]);
       __half* dst_l = a.Kl + (static_cast<long long>(h) * a.Lk + j) * D;
       store8_f16(dst_l + k0, y1);
       store8_f16(dst_l + P + k0, y2);
     }
+    if (!fin) report_status(kDevRange, 41);
   }
 }
 

@@ -101,3 +101,28 @@ def test_qwen3_8b_decode_200_steps_crossing_128k():
     _, _, res = session(w, check)
     gs = {t: g for t, _, g, _ in res}
     assert gs[71] == 4 and gs[72] == 5
+
+
+@pytest.mark.parametrize("w0", [0, 400])
+def test_force_bifocal_decode_matches_oracle(w0):
+    # BF_FLAG_FORCE_BIFOCAL runs the two-branch split-KV kernel whatever G and w0 are, as in
+    # prefill: with G == 1 (L <= w_pretrained) every pair uses the original RoPE; with w0 >= L
+    # every pair is local. Either way the result is plain RoPE attention.
+    hq, hkv, D, L = 8, 2, 128, 300
+    g = si.generator(51 + w0)
+    kc = torch.randn(L + 4, hkv, D, generator=g).to(torch.bfloat16)
+    vc = torch.randn(L + 4, hkv, D, generator=g).to(torch.bfloat16)
+    q = torch.randn(hq, D, generator=g).to(torch.bfloat16)
+    kn = torch.randn(hkv, D, generator=g).to(torch.bfloat16)
+    vn = torch.randn(hkv, D, generator=g).to(torch.bfloat16)
+    w_pre = 512 if w0 == 0 else 128  # G = 1 with w0 = 0 (all long, but the long RoPE is the original one)
+    ref_k = kc.float().double().numpy().copy()
+    ref_v = vc.float().double().numpy().copy()
+    ref_k[L - 1] = bf16_round(R.rope_keys_for_cache(kn[None].float().double().numpy(), 1e4, start=L - 1)[0])
+    ref_v[L - 1] = vn.float().double().numpy()
+    out, lse = bfl.bifocal_decode(q.cuda(), kn.cuda(), vn.cuda(), kc.cuda(), vc.cuda(), L, w0=w0, w_pretrained=w_pre,
+                                  theta=1e4, flags=bfl.FLAG_FORCE_BIFOCAL)
+    torch.cuda.synchronize()
+    assert bfl.last_device_error() == 0
+    ro, rl = R.bifocal_decode_reference(q.float().double().numpy(), ref_k, ref_v, L, w0, w_pre, 1e4, si.FREQ_INTERP)
+    assert_close(out.cpu().float().numpy(), lse.cpu().numpy(), ro, rl, f"forced decode w0={w0}")

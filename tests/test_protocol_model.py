@@ -236,3 +236,241 @@ def test_model_catches_a_missing_q_free_wait():
         except AssertionError:
             caught += 1
     assert caught > 0
+
+
+# ---------------------------------------------------------------- fused-load form
+NK3, NV2 = 3, 2  # fused form: K ring (raw tile lands, transform warps rotate it in place) and V ring
+
+
+def run_protocol_fused(sch, rnd, skip_kraw_wait=False):
+    """The fused form's protocol: the TMA producer brings raw Q, raw K tiles (ring of three) and V
+    tiles (ring of two); the transform warps rotate Q and each K tile in place once its raw bytes
+    have landed; the MMA issuer, tensor pipe and softmax groups are those of the other form, with
+    K and V on their own rings. Checks as run_protocol, plus: a raw tile never lands in a slot a
+    pending MMA reads, and the transform never touches a slot before its raw bytes have landed."""
+    nv = sch["n_long"] + sch["n_loc"]
+    has_long, has_orig = sch["n_long"] > 0, sch["n_loc"] > 0
+    reload_q = has_long and has_orig
+    v_sw = sch["n_long"]
+    kraw = [Bar(1) for _ in range(NK3)]
+    kfull = [Bar(1) for _ in range(NK3)]
+    kempty = [Bar(1) for _ in range(NK3)]
+    vfull = [Bar(1) for _ in range(NV2)]
+    vempty = [Bar(1) for _ in range(NV2)]
+    s_full, p_ready, o_done = [Bar(1), Bar(1)], [Bar(4), Bar(4)], [Bar(1), Bar(1)]
+    q_raw, q_full, q_free = Bar(1), Bar(1), Bar(1)
+    tma, pipe = [], []
+    state = {"q_readers": 0, "k_readers": [0] * NK3, "v_readers": [0] * NV2, "k_landed": [0] * NK3}
+
+    # The producer issues K two visits ahead of V (step u: K(u), then V(u - 2)), so a K fill never
+    # waits behind a V slot; the raw Q reload goes out once q_free has completed: tried at step
+    # v_sw, waited for at step v_sw + 1 (after V(v_sw - 1), which the MMA needs to get there).
+    prod = [("loadq",)]
+    for u in range(nv + 2):
+        if u < nv:
+            prod.append(("kfill", u))
+        if 2 <= u < nv + 2:
+            prod.append(("vfill", u - 2))
+        if reload_q and u == v_sw:
+            prod.append(("tryq",))
+        if reload_q and u == v_sw + 1:
+            prod.append(("waitq",))
+
+    xf = [("wait", q_raw, 0), ("rotq",), ("arrive", q_full)]
+    for v in range(nv):
+        if not skip_kraw_wait:
+            xf.append(("wait", kraw[v % NK3], (v // NK3) & 1))
+        xf += [("rotk", v), ("arrive", kfull[v % NK3])]
+        if reload_q and v == v_sw:  # K(v_sw) first, then the reloaded Q
+            xf += [("wait", q_raw, 1), ("rotq",), ("arrive", q_full)]
+
+    mma = [("wait", q_full, 0), ("wait", kfull[0], 0), ("qk", 0, 0), ("qk", 1, 0), ("commit", kempty[0])]
+    if reload_q and v_sw == 1:
+        mma.append(("commit", q_free))
+    for v in range(nv):
+        mma += [("wait", p_ready[0], v & 1), ("wait", vfull[v % NV2], (v // NV2) & 1), ("pv", 0, v)]
+        more = v + 1 < nv
+        if more:
+            if reload_q and v + 1 == v_sw:
+                mma.append(("wait", q_full, 1))
+            mma += [("wait", kfull[(v + 1) % NK3], ((v + 1) // NK3) & 1), ("qk", 0, v + 1)]
+        mma += [("wait", p_ready[1], v & 1), ("pv", 1, v), ("commit", vempty[v % NV2])]
+        if more:
+            mma += [("qk", 1, v + 1), ("commit", kempty[(v + 1) % NK3])]
+            if reload_q and v + 2 == v_sw:
+                mma.append(("commit", q_free))
+
+    def softmax_prog(x):
+        prog = []
+        for v in range(nv):
+            prog.append(("wait_s", x, v))
+            if v >= 1:
+                prog.append(("wait_o", x, v - 1))
+            prog.append(("arrive", x))
+        if nv:
+            prog.append(("wait_o", x, nv - 1))
+        return prog
+
+    progs = {"prod": prod, "xf": xf, "mma": mma, "smA": softmax_prog(0), "smB": softmax_prog(1)}
+    pc = {k: 0 for k in progs}
+
+    def land(kind, arg):
+        def go():
+            if kind == "k":
+                assert state["k_readers"][arg[0]] == 0, "raw K landed in a slot a QK^T still reads"
+                state["k_landed"][arg[0]] = arg[1] + 1
+            elif kind == "v":
+                assert state["v_readers"][arg] == 0, "V landed in a slot a PV still reads"
+            elif kind == "q":
+                assert state["q_readers"] == 0, "raw Q landed while a QK^T reads Q"
+            arg_bar.complete_tx(1)
+        arg_bar = {"k": lambda: kraw[arg[0]], "v": lambda: vfull[arg], "q": lambda: q_raw}[kind]()
+        return go
+
+    def step_prod():
+        st = progs["prod"][pc["prod"]]
+        if st[0] == "loadq":
+            q_raw.expect(1)
+            tma.append(land("q", None))
+        elif st[0] == "tryq":
+            if q_free.passed(0) and not state.get("q_reloaded"):
+                state["q_reloaded"] = True
+                q_raw.expect(1)
+                tma.append(land("q", None))
+        elif st[0] == "waitq":
+            if not state.get("q_reloaded"):
+                if not q_free.passed(0):
+                    return False
+                state["q_reloaded"] = True
+                q_raw.expect(1)
+                tma.append(land("q", None))
+        elif st[0] == "wait":
+            return st[1].passed(st[2])
+        elif st[0] == "kfill":
+            v = st[1]
+            s, use = v % NK3, v // NK3
+            if use > 0:
+                if not kempty[s].passed((use - 1) & 1):
+                    return False
+                assert kempty[s].phase == use, "K empty-slot parity alias"
+            kraw[s].expect(1)
+            tma.append(land("k", (s, v)))
+        else:
+            v = st[1]
+            s, use = v % NV2, v // NV2
+            if use > 0:
+                if not vempty[s].passed((use - 1) & 1):
+                    return False
+                assert vempty[s].phase == use, "V empty-slot parity alias"
+            vfull[s].expect(1)
+            tma.append(land("v", s))
+        return True
+
+    def step_xf():
+        st = progs["xf"][pc["xf"]]
+        if st[0] == "wait":
+            return st[1].passed(st[2])
+        if st[0] == "rotq":
+            assert state["q_readers"] == 0, "Q rotated while a QK^T reads it"
+        elif st[0] == "rotk":
+            v = st[1]
+            assert state["k_landed"][v % NK3] == v + 1, "K slot rotated before its raw tile landed"
+            assert state["k_readers"][v % NK3] == 0, "K slot rotated while a QK^T reads it"
+        else:
+            st[1].arrive()
+        return True
+
+    def step_mma():
+        st = progs["mma"][pc["mma"]]
+        if st[0] == "wait":
+            return st[1].passed(st[2])
+        if st[0] == "qk":
+            state["q_readers"] += 1
+            state["k_readers"][st[2] % NK3] += 1
+            pipe.append(("s_full", st[1], st[2]))
+        elif st[0] == "pv":
+            state["v_readers"][st[2] % NV2] += 1
+            pipe.append(("o_done", st[1], st[2]))
+        else:
+            pipe.append(("bar", st[1], None))
+        return True
+
+    def step_tensor():
+        kind, arg, v = pipe.pop(0)
+        if kind == "s_full":
+            state["q_readers"] -= 1
+            state["k_readers"][v % NK3] -= 1
+            s_full[arg].arrive()
+        elif kind == "o_done":
+            state["v_readers"][v % NV2] -= 1
+            o_done[arg].arrive()
+        else:
+            arg.arrive()
+        return True
+
+    def step_softmax(name, x):
+        st = progs[name][pc[name]]
+        if st[0] == "wait_s":
+            if not s_full[x].passed(st[2] & 1):
+                return False
+            assert s_full[x].phase == st[2] + 1, "S parity alias"
+        elif st[0] == "wait_o":
+            if not o_done[x].passed(st[2] & 1):
+                return False
+            assert o_done[x].phase >= st[2] + 1, "O parity alias"
+        else:
+            for _ in range(4):
+                p_ready[x].arrive()
+        return True
+
+    def actors():
+        out = []
+        for name, fn in (("prod", step_prod), ("xf", step_xf), ("mma", step_mma)):
+            if pc[name] < len(progs[name]):
+                out.append((name, fn))
+        if tma:
+            out.append(("tma", lambda: (tma.pop(rnd.randrange(len(tma)))(), True)[1]))
+        if pipe:
+            out.append(("tensor", step_tensor))
+        for name, x in (("smA", 0), ("smB", 1)):
+            if pc[name] < len(progs[name]):
+                out.append((name, lambda name=name, x=x: step_softmax(name, x)))
+        return out
+
+    while True:
+        acts = actors()
+        if not acts:
+            return True
+        rnd.shuffle(acts)
+        for name, fn in acts:
+            if fn():
+                if name in pc:
+                    pc[name] += 1
+                break
+        else:
+            raise AssertionError(f"deadlock at {pc}")
+
+
+@pytest.mark.parametrize("Lq,q_off,w0,kind", CASES)
+def test_fused_protocol_completes_without_aliasing(Lq, q_off, w0, kind):
+    rnd = random.Random(Lq * 17 + q_off + w0)
+    n_qt = (Lq + BM - 1) // BM
+    for qt in range(n_qt):
+        i0 = q_off + qt * BM
+        n_kt = (min(i0 + BM, q_off + Lq) + BN - 1) // BN
+        sch = schedule(i0, n_kt, w0, kind)
+        for _ in range(2):
+            assert run_protocol_fused(sch, rnd) is True
+
+
+def test_fused_model_catches_a_missing_raw_wait():
+    # planted mistake: the transform warps rotate a K slot without waiting for its raw tile
+    sch = schedule(2048, 17, 300, "bifocal")
+    rnd = random.Random(11)
+    caught = 0
+    for _ in range(100):
+        try:
+            run_protocol_fused(sch, rnd, skip_kraw_wait=True)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
