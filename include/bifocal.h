@@ -63,8 +63,12 @@ typedef enum {
   BF_ERR_TIMEOUT = 4,      /* a device-side bounded wait expired (reported by bifocal_last_device_error) */
   BF_ERR_WORKSPACE = 5,    /* workspace missing, misaligned or smaller than *_workspace_size */
   BF_ERR_NO_DEVICE = 6,    /* no CUDA device, or the device is not sm_100 */
-  BF_ERR_RANGE = 7         /* an fp16 QK^T operand (a rotated query or key) was not finite once rounded to
+  BF_ERR_RANGE = 7,        /* an fp16 QK^T operand (a rotated query or key) was not finite once rounded to
                               fp16 (|x| >= 65520, inf or NaN), so the result is not trustworthy (reported by
+                              bifocal_last_device_error) */
+  BF_ERR_INDEX = 8         /* an index the kernels read from device memory (a sequence length outside
+                              [1, max_len], a block-table entry outside [0, pool_pages)) was out of range; the
+                              cache rows it would have addressed were neither read nor written (reported by
                               bifocal_last_device_error) */
 } bf_status_t;
 
@@ -304,13 +308,19 @@ BF_API const char* bifocal_status_string(int32_t status);
  *   - a bounded wait expired (a producer never delivered, or a wait ran past the limit): BF_ERR_TIMEOUT;
  *   - an fp16 QK^T operand (a query or key after RoPE or the correction rotation, or a cached
  *     bf16 key converted to fp16) was not finite once rounded to fp16 (|x| >= 65520, inf or
- *     NaN): BF_ERR_RANGE. The decode kernel detects it as a non-finite score of a valid key.
- * Synchronises `stream` first. Returns BF_OK, BF_ERR_TIMEOUT, BF_ERR_RANGE or BF_ERR_CUDA. */
+ *     NaN): BF_ERR_RANGE. The decode kernel detects it as a non-finite running max or sum;
+ *   - a sequence length or block-table entry read from device memory by the paged entry points
+ *     was out of range: BF_ERR_INDEX. The kernels skip every cache row it would address (no
+ *     append, no pool write, its key tiles read as zeros) and a paged decode writes NaN as the
+ *     output of a sequence whose length is out of range.
+ * Synchronises `stream` first. Returns BF_OK, BF_ERR_TIMEOUT, BF_ERR_RANGE, BF_ERR_INDEX or
+ * BF_ERR_CUDA. */
 BF_API bf_status_t bifocal_last_device_error(void* stream);
 
 /* The raw device status word (not cleared): 0, or code | (site << 8) for the first event, where
- * code is 1 (a bounded wait expired) or 2 (an fp16 operand out of range) and `site` numbers the
- * wait or the check in the kernel source. Synchronises the device. Returns -1 on a CUDA error. */
+ * code is 1 (a bounded wait expired), 2 (an fp16 operand out of range) or 3 (a device-side index
+ * out of range) and `site` numbers the wait or the check in the kernel source. Synchronises the
+ * device. Returns -1 on a CUDA error. */
 BF_API int32_t bifocal_device_status_word(void);
 
 /* Test-only fault injection for the failure-detection tests. Not needed by any caller of the
@@ -320,8 +330,8 @@ BF_API int32_t bifocal_device_status_word(void);
  *        never issues K/V fill number `arg` (no expect_tx, no copy), so the MMA issuer's wait for
  *        it can only expire: the CTA gives up, every role leaves through the normal teardown
  *        (no copy in flight, tensor memory freed) and the status word reports the wait's site.
- *   kind BF_FAULT_DECODE_SKIP_STAGE: in the split-KV decode kernel, the producer of CTA 0 never
- *        issues stage `arg`; the consumer warps' wait for it expires likewise.
+ *   kind BF_FAULT_DECODE_SKIP_STAGE: in the split-KV decode kernel, the producer of CTA 0 issues
+ *        no stage from stage `arg` on; the consumer warps' wait for stage `arg` expires likewise.
  *   wait_limit_ns: the limit of every bounded wait in ns; 0 restores the default of 2 s. A wait
  *        consults it only after 20 ms, so a smaller limit acts as 20 ms.
  * Synchronises the device before and after setting the controls. Returns BF_ERR_INVALID for an

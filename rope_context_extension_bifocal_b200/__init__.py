@@ -17,7 +17,7 @@ __all__ = [
     "BifocalError", "FREQ_INTERP", "POS_ALIAS", "FLAG_FORCE_BIFOCAL", "FLAG_MMA_SYNC", "FLAG_WINDOW", "FLAG_FUSED_ROPE", "Params", "lib", "lib_path",
     "bifocal_factor", "bifocal_prefill", "bifocal_prefill_rope", "bifocal_prefill_attention", "rope_causal_prefill", "bifocal_prefill_chunk_paged", "bifocal_decode", "bifocal_decode_noalloc", "rope_causal_decode",
     "prefill_workspace_size", "decode_workspace_size", "last_device_error", "build_info", "test_set_fault",
-    "STATUS_TIMEOUT", "STATUS_RANGE", "FAULT_NONE", "FAULT_PREFILL_SKIP_FILL", "FAULT_DECODE_SKIP_STAGE",
+    "STATUS_TIMEOUT", "STATUS_RANGE", "STATUS_INDEX", "FAULT_NONE", "FAULT_PREFILL_SKIP_FILL", "FAULT_DECODE_SKIP_STAGE",
 ]
 
 FREQ_INTERP = "freq_interp"
@@ -28,7 +28,7 @@ FLAG_MMA_SYNC = 2
 FLAG_WINDOW = 4
 FLAG_FUSED_ROPE = 8
 DTYPE_BF16, DTYPE_FP32 = 0, 1
-STATUS_TIMEOUT, STATUS_RANGE = 4, 7
+STATUS_TIMEOUT, STATUS_RANGE, STATUS_INDEX = 4, 7, 8
 FAULT_NONE, FAULT_PREFILL_SKIP_FILL, FAULT_DECODE_SKIP_STAGE = 0, 1, 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -363,13 +363,15 @@ def rope_causal_decode(q, k_new, v_new, kcache, vcache, L: int, *, theta: float,
 
 
 def device_status_word() -> int:
-    """Raw device status word: 0, or 1 | (site << 8) of the first expired bounded wait."""
+    """Raw device status word: 0, or code | (site << 8) of the first device-side event (code 1: a
+    bounded wait expired, 2: an fp16 operand out of range, 3: a device-side index out of range)."""
     return int(_lib().bifocal_device_status_word())
 
 
 def last_device_error(stream=None) -> int:
     """Status of the device-side checks since the last call, then cleared: 0, STATUS_TIMEOUT (a
-    bounded wait expired) or STATUS_RANGE (an fp16 QK^T operand was out of range)."""
+    bounded wait expired), STATUS_RANGE (an fp16 QK^T operand was out of range) or STATUS_INDEX (a
+    sequence length or block-table entry in device memory was out of range)."""
     return int(_lib().bifocal_last_device_error(_stream(stream)))
 
 

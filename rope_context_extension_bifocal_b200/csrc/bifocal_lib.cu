@@ -23,6 +23,12 @@ using bf16 = __nv_bfloat16;
 
 constexpr int kMaxSplits = 320;  // split-KV partials reserved in the decode workspace
 
+// Test-only fault injection (bifocal_test_set_fault), passed to the kernels as arguments: one
+// more than the fill of the prefill producer / the stage of the decode producer that CTA 0 never
+// issues; 0 = off (so an argument block cleared to zero never skips anything).
+int g_test_skip_fill = 0;
+int g_test_skip_stage = 0;
+
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct Rope {
@@ -323,6 +329,7 @@ bf_status_t fused_attention(int kind, const void* q, const void* ksrc, bool cach
   ta.q_off = q_off;
   ta.Lq = Lq;
   ta.scale_log2 = scale_log2(p);
+  ta.test_skip_fill = g_test_skip_fill;
   ta.src.cache = cache ? 1 : 0;
   ta.src.mode = p->mode;
   ta.src.G = G;
@@ -364,7 +371,6 @@ bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtyp
   aa.w0 = plan.kind != bf::tc2::KIND_PLAIN ? p->w0 : L;
   aa.scale_log2 = scale_log2(p);
   cudaError_t e;
-  const int g = p->hq / p->hkv;
   if (tc2_path(p)) {
     // tcgen05 ping-pong path: two heads of one GQA group per CTA
     bf::Tc2Args ta;
@@ -383,7 +389,8 @@ bf_status_t prefill_attention_impl(bool bifocal_api, const void* v, int32_t dtyp
     ta.q_off = 0;
     ta.Lq = L;
     ta.scale_log2 = aa.scale_log2;
-      constexpr int smem = bf::attn_tc2_smem_bytes();
+    ta.test_skip_fill = g_test_skip_fill;
+    constexpr int smem = bf::attn_tc2_smem_bytes();
     const long long n_cta = static_cast<long long>((L + bf::tc::BM - 1) / bf::tc::BM) * (p->hq / 2) * batch;
     if (n_cta > 0x7fffffffLL) return BF_ERR_UNSUPPORTED;
     auto kern = plan.kind == bf::tc2::KIND_BIFOCAL  ? bf::attn_tc2_kernel<bf::tc2::KIND_BIFOCAL, false>
@@ -568,6 +575,7 @@ bf_status_t chunk_impl(const void* q, const void* k, const void* v, int32_t dtyp
   ta.q_off = P0;
   ta.Lq = C;
   ta.scale_log2 = scale_log2(p);
+  ta.test_skip_fill = g_test_skip_fill;
   constexpr int smem = bf::attn_tc2_smem_bytes();
   const long long n_cta = static_cast<long long>((C + bf::tc::BM - 1) / bf::tc::BM) * (p->hq / 2);
   auto kern = kind == bf::tc2::KIND_BIFOCAL  ? bf::attn_tc2_kernel<bf::tc2::KIND_BIFOCAL, false>
@@ -605,10 +613,54 @@ struct DecodeLayout {
   size_t part_o, part_ml, total;
 };
 
+// The split-KV partial kernel; the test instantiation only while a skipped stage is armed.
+template <int D, bool TEST>
+cudaError_t launch_partial_t(dim3 grid, cudaStream_t st, const bf::DecodeArgs& da) {
+  constexpr int smem = bf::decode_smem_bytes<D>();
+  cudaError_t e = cudaFuncSetAttribute(bf::decode_partial_kernel<D, TEST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(bf::decode_partial_kernel<D, TEST>, grid, dim3(bf::decode_threads<D>()), smem, st, da);
+}
+
+cudaError_t launch_partial(int D, dim3 grid, cudaStream_t st, const bf::DecodeArgs& da) {
+  const bool test = da.test_skip_stage > 0;
+  if (D == 128) return test ? launch_partial_t<128, true>(grid, st, da) : launch_partial_t<128, false>(grid, st, da);
+  return test ? launch_partial_t<64, true>(grid, st, da) : launch_partial_t<64, false>(grid, st, da);
+}
+
+// The combine (PDL-chained to the partial kernel), with the smallest load batch NB that covers
+// a warp's share of the at most n_split partials per head in one pass.
+template <int D, int NB>
+cudaError_t launch_combine_t(dim3 grid, cudaStream_t st, const float* po, const float* pml, int n_split, int hq,
+                             bf16* out, float* lse, const int* seq_lens, int split_len, int stride, int max_len) {
+  return launch_pdl(bf::decode_combine_kernel<D, NB>, grid, dim3(32 * bf::COMBINE_WARPS), 0, st, po, pml, n_split,
+                    hq, out, lse, seq_lens, split_len, stride, max_len);
+}
+
+template <int D>
+cudaError_t launch_combine_d(dim3 grid, cudaStream_t st, const float* po, const float* pml, int n_split, int hq,
+                             bf16* out, float* lse, const int* seq_lens, int split_len, int stride, int max_len) {
+  const int per_warp = (n_split + bf::COMBINE_WARPS - 1) / bf::COMBINE_WARPS;
+  if (per_warp <= 2)
+    return launch_combine_t<D, 2>(grid, st, po, pml, n_split, hq, out, lse, seq_lens, split_len, stride, max_len);
+  if (per_warp <= 4)
+    return launch_combine_t<D, 4>(grid, st, po, pml, n_split, hq, out, lse, seq_lens, split_len, stride, max_len);
+  if (per_warp <= 8)
+    return launch_combine_t<D, 8>(grid, st, po, pml, n_split, hq, out, lse, seq_lens, split_len, stride, max_len);
+  return launch_combine_t<D, 16>(grid, st, po, pml, n_split, hq, out, lse, seq_lens, split_len, stride, max_len);
+}
+
+cudaError_t launch_combine(int D, dim3 grid, cudaStream_t st, const float* po, const float* pml, int n_split, int hq,
+                           bf16* out, float* lse, const int* seq_lens, int split_len, int stride, int max_len) {
+  return D == 128 ? launch_combine_d<128>(grid, st, po, pml, n_split, hq, out, lse, seq_lens, split_len, stride, max_len)
+                  : launch_combine_d<64>(grid, st, po, pml, n_split, hq, out, lse, seq_lens, split_len, stride, max_len);
+}
+
 DecodeLayout decode_layout(int L_max, const bf_params_t* p) {
   DecodeLayout w{};
-  // two partials (one per consumer warp of a kv head) per CTA split
-  const int splits = 2 * std::min(kMaxSplits, (L_max + bf::dec::KB - 1) / bf::dec::KB);
+  // one partial per CTA split (the two consumer warps of a kv head merge theirs in the CTA)
+  const int splits = std::min(kMaxSplits, (L_max + bf::dec::KB - 1) / bf::dec::KB);
   w.part_o = 0;
   w.part_ml = align256(static_cast<size_t>(splits) * p->hq * p->head_dim * 4);
   w.total = w.part_ml + align256(static_cast<size_t>(splits) * p->hq * 2 * 4);
@@ -648,11 +700,10 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
   ap.hkv = p->hkv;
   ap.p = L - 1;
   std::memcpy(ap.omega, rope.omega, sizeof(ap.omega));
-  if (D == 128)
-    bf::decode_append_kernel<128><<<p->hkv, 32, 0, st>>>(ap);
-  else
-    bf::decode_append_kernel<64><<<p->hkv, 32, 0, st>>>(ap);
-  if (cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
+  // launched early (PDL): it waits in the kernel for whatever ran before it on the stream
+  cudaError_t ea = D == 128 ? launch_pdl(bf::decode_append_kernel<128>, dim3(p->hkv), dim3(32), 0, st, ap)
+                            : launch_pdl(bf::decode_append_kernel<64>, dim3(p->hkv), dim3(32), 0, st, ap);
+  if (ea != cudaSuccess) return BF_ERR_CUDA;
 
   // 2. split-KV partials
   bf::DecodeArgs da;
@@ -681,38 +732,19 @@ bf_status_t decode_impl(bool bifocal_api, const void* q, const void* k_new, cons
   da.split_len = split_len;
   da.n_split = n_split;
   da.scale_log2 = scale_log2(p);
+  da.test_skip_stage = g_test_skip_stage;
   std::memcpy(da.omega, rope.omega, sizeof(da.omega));
   std::memcpy(da.omega_long, rope.omega_long, sizeof(da.omega_long));
   std::memcpy(da.omega_corr, rope.omega_corr, sizeof(da.omega_corr));
   const dim3 grid(n_split, head_groups);
   cudaError_t e;
   // the partial and combine kernels overlap their launch with the kernel before them
-  if (D == 128) {
-    constexpr int smem = bf::decode_smem_bytes<128>();
-    e = cudaFuncSetAttribute(bf::decode_partial_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess)
-      e = launch_pdl(bf::decode_partial_kernel<128>, grid, dim3(bf::decode_threads<128>()), smem, st, da);
-  } else {
-    constexpr int smem = bf::decode_smem_bytes<64>();
-    e = cudaFuncSetAttribute(bf::decode_partial_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess)
-      e = launch_pdl(bf::decode_partial_kernel<64>, grid, dim3(bf::decode_threads<64>()), smem, st, da);
-  }
+  e = launch_partial(D, grid, st, da);
   if (e != cudaSuccess) return BF_ERR_CUDA;
 
   // 3. combine
-  const float* po = da.part_o;
-  const float* pml = da.part_ml;
-  const int nparts = 2 * n_split;
-  const int hq = p->hq;
-  bf16* o16 = static_cast<bf16*>(out);
-  const dim3 cblock(32 * bf::COMBINE_WARPS);
-  if (D == 128)
-    e = launch_pdl(bf::decode_combine_kernel<128>, dim3(p->hq, 128 / 32), cblock, 0, st, po, pml, nparts, hq, o16, lse,
-                   static_cast<const int*>(nullptr), 0, 0);
-  else
-    e = launch_pdl(bf::decode_combine_kernel<64>, dim3(p->hq, 64 / 32), cblock, 0, st, po, pml, nparts, hq, o16, lse,
-                   static_cast<const int*>(nullptr), 0, 0);
+  e = launch_combine(D, dim3(p->hq, D / 32), st, da.part_o, da.part_ml, n_split, p->hq, static_cast<bf16*>(out), lse,
+                     nullptr, 0, 0, 0);
   return e == cudaSuccess ? BF_OK : BF_ERR_CUDA;
 }
 
@@ -782,7 +814,7 @@ void* noalloc_scratch_ptr() {
 
 // ------------------------------------------------------------------ batched decode over a paged cache
 // Partial rows per sequence: two per split, splits <= min(kMaxSplits, ceil(max_len / KB)).
-int paged_parts_stride(int max_len) { return 2 * std::min(kMaxSplits, (max_len + bf::dec::KB - 1) / bf::dec::KB); }
+int paged_parts_stride(int max_len) { return std::min(kMaxSplits, (max_len + bf::dec::KB - 1) / bf::dec::KB); }
 
 size_t paged_workspace(int batch, int max_len, const bf_params_t* p) {
   const size_t rows = static_cast<size_t>(batch) * paged_parts_stride(max_len) * p->hq;
@@ -828,12 +860,12 @@ bf_status_t decode_paged_impl(const void* q, const void* k_new, const void* v_ne
   ap.block_table = block_table;
   ap.max_pages = max_pages;
   ap.page_size = page_size;
+  ap.pool_pages = pool_pages;
+  ap.max_len = max_len;
   std::memcpy(ap.omega, rope.omega, sizeof(ap.omega));
-  if (D == 128)
-    bf::decode_append_kernel<128><<<dim3(p->hkv, batch), 32, 0, st>>>(ap);
-  else
-    bf::decode_append_kernel<64><<<dim3(p->hkv, batch), 32, 0, st>>>(ap);
-  if (cudaGetLastError() != cudaSuccess) return BF_ERR_CUDA;
+  cudaError_t ea = D == 128 ? launch_pdl(bf::decode_append_kernel<128>, dim3(p->hkv, batch), dim3(32), 0, st, ap)
+                            : launch_pdl(bf::decode_append_kernel<64>, dim3(p->hkv, batch), dim3(32), 0, st, ap);
+  if (ea != cudaSuccess) return BF_ERR_CUDA;
 
   // 2. split-KV partials: one split length for the batch (from max_len), a grid of about one
   //    CTA per SM in total; CTAs past a shorter sequence's end leave at once
@@ -868,32 +900,16 @@ bf_status_t decode_paged_impl(const void* q, const void* k_new, const void* v_ne
   da.w_pretrained = p->w_pretrained;
   da.force_bifocal = (p->flags & BF_FLAG_FORCE_BIFOCAL) ? 1 : 0;
   da.parts_stride = stride;
+  da.pool_pages = pool_pages;
+  da.test_skip_stage = g_test_skip_stage;
   const dim3 grid(n_split, head_groups, batch);
   cudaError_t e;
-  if (D == 128) {
-    constexpr int smem = bf::decode_smem_bytes<128>();
-    e = cudaFuncSetAttribute(bf::decode_partial_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess)
-      e = launch_pdl(bf::decode_partial_kernel<128>, grid, dim3(bf::decode_threads<128>()), smem, st, da);
-  } else {
-    constexpr int smem = bf::decode_smem_bytes<64>();
-    e = cudaFuncSetAttribute(bf::decode_partial_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess)
-      e = launch_pdl(bf::decode_partial_kernel<64>, grid, dim3(bf::decode_threads<64>()), smem, st, da);
-  }
+  e = launch_partial(D, grid, st, da);
   if (e != cudaSuccess) return BF_ERR_CUDA;
 
   // 3. combine per sequence
-  const dim3 cblock(32 * bf::COMBINE_WARPS);
-  bf16* o16 = static_cast<bf16*>(out);
-  if (D == 128)
-    e = launch_pdl(bf::decode_combine_kernel<128>, dim3(p->hq, 128 / 32, batch), cblock, 0, st,
-                   static_cast<const float*>(part_o), static_cast<const float*>(part_ml), 2 * n_split, p->hq, o16,
-                   lse, static_cast<const int*>(seq_lens), split_len, stride);
-  else
-    e = launch_pdl(bf::decode_combine_kernel<64>, dim3(p->hq, 64 / 32, batch), cblock, 0, st,
-                   static_cast<const float*>(part_o), static_cast<const float*>(part_ml), 2 * n_split, p->hq, o16,
-                   lse, static_cast<const int*>(seq_lens), split_len, stride);
+  e = launch_combine(D, dim3(p->hq, D / 32, batch), st, part_o, part_ml, n_split, p->hq, static_cast<bf16*>(out), lse,
+                     seq_lens, split_len, stride, max_len);
   return e == cudaSuccess ? BF_OK : BF_ERR_CUDA;
 }
 
@@ -952,6 +968,7 @@ bf_status_t chunk_paged_impl(const void* q, const void* k, const void* v, int32_
   pa.block_table = block_table;
   pa.max_pages = max_pages;
   pa.page_size = page_size;
+  pa.pool_pages = pool_pages;
   int row = 0;
   for (int i = 0; i < batch; ++i) {
     pa.seq_id[i] = i;
@@ -983,12 +1000,14 @@ bf_status_t chunk_paged_impl(const void* q, const void* k, const void* v, int32_
   ta.src.mode = p->mode;
   ta.src.G = 1;
   std::memcpy(ta.src.omega, rope.omega, sizeof(ta.src.omega));
+  ta.test_skip_fill = g_test_skip_fill;
   ta.nseq = batch;
   ta.total_rows = T;
   ta.block_table = block_table;
   ta.max_pages = max_pages;
   ta.page_size = page_size;
   ta.seg_rows = seg;
+  ta.pool_pages = pool_pages;
   int tiles = 0;
   for (int si = 0; si < batch; ++si) {
     const int i = order[si];
@@ -1131,6 +1150,7 @@ const char* bifocal_status_string(int32_t status) {
     case BF_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case BF_ERR_NO_DEVICE: return "no suitable CUDA device";
     case BF_ERR_RANGE: return "an fp16 QK^T operand was not finite after rounding (|x| >= 65520, inf or NaN)";
+    case BF_ERR_INDEX: return "a sequence length or block-table entry in device memory was out of range";
     default: return "unknown status";
   }
 }
@@ -1142,22 +1162,23 @@ bf_status_t bifocal_last_device_error(void* stream) {
   if (v == 0) return BF_OK;
   const int zero = 0;
   if (cudaMemcpyToSymbol(bf::g_device_status, &zero, sizeof(int)) != cudaSuccess) return BF_ERR_CUDA;
-  return (v & 0xff) == bf::kDevRange ? BF_ERR_RANGE : BF_ERR_TIMEOUT;
+  switch (v & 0xff) {
+    case bf::kDevRange: return BF_ERR_RANGE;
+    case bf::kDevIndex: return BF_ERR_INDEX;
+    default: return BF_ERR_TIMEOUT;
+  }
 }
 
 bf_status_t bifocal_test_set_fault(int32_t kind, int32_t arg, int64_t wait_limit_ns) {
   if (kind < BF_FAULT_NONE || kind > BF_FAULT_DECODE_SKIP_STAGE || wait_limit_ns < 0) return BF_ERR_INVALID;
   if (kind != BF_FAULT_NONE && arg < 0) return BF_ERR_INVALID;
   if (cudaDeviceSynchronize() != cudaSuccess) return BF_ERR_CUDA;  // no launch in flight sees a half-set control
-  const int off = -1;
-  const int pre = kind == BF_FAULT_PREFILL_SKIP_FILL ? arg : off;
-  const int dec = kind == BF_FAULT_DECODE_SKIP_STAGE ? arg : off;
   const unsigned long long lim = wait_limit_ns > 0 ? static_cast<unsigned long long>(wait_limit_ns) : 2000000000ull;
-  if (cudaMemcpyToSymbol(bf::g_skip_fill_prefill, &pre, sizeof(int)) != cudaSuccess ||
-      cudaMemcpyToSymbol(bf::g_skip_stage_decode, &dec, sizeof(int)) != cudaSuccess ||
-      cudaMemcpyToSymbol(bf::g_wait_limit_ns, &lim, sizeof(lim)) != cudaSuccess ||
+  if (cudaMemcpyToSymbol(bf::g_wait_limit_ns, &lim, sizeof(lim)) != cudaSuccess ||
       cudaDeviceSynchronize() != cudaSuccess)
     return BF_ERR_CUDA;
+  g_test_skip_fill = kind == BF_FAULT_PREFILL_SKIP_FILL ? arg + 1 : 0;
+  g_test_skip_stage = kind == BF_FAULT_DECODE_SKIP_STAGE ? arg + 1 : 0;
   return BF_OK;
 }
 

@@ -15,9 +15,12 @@ namespace bf {
 //   kDevTimeout | site << 8   a bounded wait gave up (site numbers the wait in the source)
 //   kDevRange   | site << 8   an operand of the fp16 QK^T product was not finite after
 //                             rounding to fp16 (|x| >= 65520, inf or NaN)
+//   kDevIndex   | site << 8   an index read from device memory (a sequence length or a
+//                             block-table entry) was out of range; the reads and writes it
+//                             would have addressed were skipped
 // Read and cleared by bifocal_last_device_error().
 // ---------------------------------------------------------------------------------
-enum : int { kDevOk = 0, kDevTimeout = 1, kDevRange = 2 };
+enum : int { kDevOk = 0, kDevTimeout = 1, kDevRange = 2, kDevIndex = 3 };
 __device__ int g_device_status = 0;
 
 // Wall-clock limit of every bounded wait, in ns (2 s; a test may shorten it through
@@ -26,13 +29,6 @@ __device__ int g_device_status = 0;
 // polling loops of normal operation compare against a constant and never touch global memory.
 __device__ unsigned long long g_wait_limit_ns = 2000000000ull;
 constexpr unsigned long long kWaitFloorNs = 20000000ull;
-
-// Test-only fault injection, off (-1) unless a test sets it through bifocal_test_set_fault:
-// the producer of CTA 0 skips one whole fill (no expect_tx, no copy), so the wait for it
-// can only expire. Prefill: fill number g_skip_fill_prefill of the K/V ring; decode:
-// stage number g_skip_stage_decode of the split-KV kernel.
-__device__ int g_skip_fill_prefill = -1;
-__device__ int g_skip_stage_decode = -1;
 
 __device__ __forceinline__ void report_status(int code, int where) {
   if (*reinterpret_cast<volatile int*>(&g_device_status) == kDevOk) atomicCAS(&g_device_status, kDevOk, code | (where << 8));
@@ -219,6 +215,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, int whe
   }
   report_timeout(where);
   return false;
+}
+
+// Bounded wait for a thread that has nothing else to do until the phase completes (a
+// producer waiting for its last copies before the CTA exits): sleeps between polls, so it
+// takes no issue slots from the warps still working on the same SM sub-partition.
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t* bar, uint32_t phase, int where) {
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, phase)) {
+    __nanosleep(500);
+    const uint64_t el = global_ns() - t0;
+    if (el > kWaitFloorNs && el > *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns)) {
+      report_timeout(where);
+      return false;
+    }
+  }
+  return true;
 }
 
 // Same, but also gives up as soon as *abort is set (by any warp of the CTA), and sets it

@@ -51,7 +51,9 @@ struct DecodeArgs {
   const int* seq_lens;
   const int* block_table;
   int max_pages, page_size, w_pretrained, force_bifocal;
+  int pool_pages;    // block-table entries must lie in [0, pool_pages); lengths in [1, L = max_len]
   int parts_stride;  // partial rows reserved per sequence
+  int test_skip_stage;  // test only (bifocal_test_set_fault): 1 + the stage CTA 0's producer never issues; 0 = off
 };
 
 // 128-byte swizzle of TMA SWIZZLE_128B: 16-byte chunk c of row r sits at chunk c ^ (r & 7).
@@ -59,7 +61,10 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
   return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int D>
+// TEST = true is the instantiation launched only while bifocal_test_set_fault has armed a
+// skipped stage: its producer stops issuing at that stage in CTA 0. The normal instantiation has
+// no trace of it (a changed loop bound in the producer cost up to 20 us per step).
+template <int D, bool TEST>
 __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
   using namespace dec;
   constexpr int P = D / 2;
@@ -81,6 +86,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   uint64_t* full = reinterpret_cast<uint64_t*>(sCS + NST * STAGE_CS);
   uint64_t* empty = full + NST;
   uint64_t* tbl = empty + NST;
+  uint8_t* xch = reinterpret_cast<uint8_t*>(tbl + NST);  // [HPC][4 * MT + 2][32] floats: warp-pair exchange
   __shared__ int s_abort;  // set when a bounded wait expires: later waits return at once
 
   pdl_launch_dependents();  // the combine may start its prologue; it waits for this grid's writes
@@ -91,6 +97,10 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   const bool paged = a.seq_lens != nullptr;
   const int bz = paged ? static_cast<int>(blockIdx.z) : 0;
   const int L = paged ? a.seq_lens[bz] : a.L;
+  if (paged && (L < 1 || L > a.L)) {  // a length the batch's tables and partial rows cannot hold (a.L = max_len)
+    if (threadIdx.x == 0) report_status(kDevIndex, 52);
+    return;
+  }
   const int G = paged ? (L <= a.w_pretrained ? 1 : (L + a.w_pretrained - 1) / a.w_pretrained) : a.G;
   const bool bifocal = paged ? (a.force_bifocal || (G > 1 && a.w0 < L)) : (a.bifocal != 0);
   const int p = L - 1;
@@ -121,22 +131,36 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
       prefetch_tensormap(&a.kmap);
       prefetch_tensormap(&a.vmap);
       const uint32_t bytes = 2u * nheads * HALVES * HEAD_TILE;
-      int skip = -1;  // test only: a volatile read inside the branch, so no other CTA waits for the load
-      if ((blockIdx.x | blockIdx.y | blockIdx.z) == 0) skip = *reinterpret_cast<volatile int*>(&g_skip_stage_decode);
+      // test instantiation only: CTA 0 issues no stage from test_skip_stage - 1 on
+      const int n_issue = (TEST && (blockIdx.x | blockIdx.y | blockIdx.z) == 0) ? min(nstage, a.test_skip_stage - 1)
+                                                                                 : nstage;
       uint32_t used = 0, par = 0;  // per slot: has a fill been issued, parity of the fills issued
-      for (int s = 0; s < nstage; ++s) {
+      // paged: the block-table entry of the current page and, loaded one page ahead, of the next
+      // (the stages of a split walk its pages in order, so the load has a page of stages to land)
+      int cur_idx = -1, cur_row0 = 0;
+      int nxt_pg = paged ? a.block_table[static_cast<long long>(bz) * a.max_pages + jbeg / a.page_size] : 0;
+      for (int s = 0; s < n_issue; ++s) {
         const int st = s % NST;
         if (s >= NST && !mbar_wait_abortable(&empty[st], ((s / NST) - 1) & 1, 1, &s_abort)) break;
-        if (*reinterpret_cast<volatile int*>(&s_abort)) break;  // a consumer gave up: issue nothing more
-        if (s == skip) continue;
         const int j0 = jbeg + s * KB;
         // Only row p (the new token) comes from the append kernel; every other row was in the
         // cache before this step, so only the stage holding p waits for that grid.
         if (j0 + KB > p) pdl_wait();
         // pool row of logical key j0 (pages hold a multiple of KB keys, so a stage is one page's)
-        const int row = paged ? a.block_table[static_cast<long long>(bz) * a.max_pages + j0 / a.page_size] * a.page_size +
-                                    j0 % a.page_size
-                              : j0;
+        int row = j0;
+        if (paged) {
+          const int idx = j0 / a.page_size;
+          if (idx != cur_idx) {
+            const int pg = nxt_pg;
+            cur_idx = idx;
+            nxt_pg = idx + 1 < a.max_pages ? a.block_table[static_cast<long long>(bz) * a.max_pages + idx + 1] : 0;
+            const bool pg_ok = pg >= 0 && pg < a.pool_pages;
+            if (!pg_ok) report_status(kDevIndex, 53);
+            // a bad entry loads stages that start just past the pool's last row: TMA fills them with zeros
+            cur_row0 = pg_ok ? pg * a.page_size : a.pool_pages * a.page_size - j0 % a.page_size;
+          }
+          row = cur_row0 + j0 % a.page_size;
+        }
         mbar_arrive_expect_tx(&full[st], bytes);
         for (int hh = 0; hh < nheads; ++hh)
           for (int hf = 0; hf < HALVES; ++hf) {
@@ -147,11 +171,15 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
         used |= 1u << st;
         par ^= 1u << st;
       }
-      // Every copy issued must have landed before the CTA may exit. The consumers wait for each
-      // stage they read, but after an expired wait they stop waiting, so the producer itself
-      // waits for the last fill of every slot (bounded, not abortable).
-      for (int st = 0; st < NST; ++st)
-        if (used & (1u << st)) mbar_wait(&full[st], ((par >> st) & 1u) ^ 1u, 4);
+      // Every copy issued must land before the CTA exits. The consumers wait for every stage
+      // they read, so normally nothing is in flight when they finish and the producer leaves at
+      // once (holding this warp until the consumers were done cost 2-6 us per decode step). If a
+      // wait expired before the producer got here, it waits (bounded) for the last copy it issued
+      // into each slot. An expiry after it left can only come from a copy that did not land
+      // within the limit, which no wait could repair.
+      if (*reinterpret_cast<volatile int*>(&s_abort))
+        for (int st = 0; st < NST; ++st)
+          if (used & (1u << st)) mbar_wait_sleepy(&full[st], ((par >> st) & 1u) ^ 1u, 4);
     }
     return;
   }
@@ -223,6 +251,7 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   // query fragments (rows 0..g-1 = the g query heads of this kv head) under both RoPE forms,
   // fp16, in the m16n8k16 A layout: qa_*[kc] = {a0, a2} of k-chunk kc (rows 8..15 are zero)
   uint32_t qa_o[KC][2], qa_l[KC][2];
+  bool q_fin = true;  // the rotated query fragments fit fp16
   {
     const bool row_ok = g8 < g;
     const __nv_bfloat16* qrow = a.q + (static_cast<long long>(bz) * a.hq + kvh * g + (row_ok ? g8 : 0)) * D;
@@ -251,9 +280,8 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
           xl[e] = x * c - y * sn;
           yl[e] = y * c + x * sn;
         }
-        if (!(f16_ok(xo[0]) & f16_ok(xo[1]) & f16_ok(yo[0]) & f16_ok(yo[1]) & f16_ok(xl[0]) & f16_ok(xl[1]) &
-              f16_ok(yl[0]) & f16_ok(yl[1])))
-          report_status(kDevRange, 42);
+        q_fin &= f16_ok(xo[0]) & f16_ok(xo[1]) & f16_ok(yo[0]) & f16_ok(yo[1]) & f16_ok(xl[0]) & f16_ok(xl[1]) &
+                 f16_ok(yl[0]) & f16_ok(yl[1]);
         qa_o[kc][sub] = pack_f16x2(xo[0], xo[1]);
         qa_o[kc + KCP][sub] = pack_f16x2(yo[0], yo[1]);
         qa_l[kc][sub] = pack_f16x2(xl[0], xl[1]);
@@ -266,7 +294,6 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
 #pragma unroll
   for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m_r = -INFINITY, l_r = 0.f;  // softmax state of query row g8 (S layout)
-  bool scores_fin = true;            // every score of a valid key came out finite (fp16 operands in range)
 
   for (int s = 0; s < nstage; ++s) {
     const int st = s % NST;
@@ -326,7 +353,6 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
       // An fp16 operand that overflowed (|x| >= 65520 rounds to inf) or a NaN key makes the
       // score inf or NaN (the padding query rows are zero: 0 * inf = NaN), so one test per
       // score covers every key operand of the stage.
-      if (j < jend) scores_fin &= fabsf(x) < INFINITY;
       x *= a.scale_log2;
       if (j >= jend) x = -INFINITY;
       sc[e] = x;
@@ -382,11 +408,49 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
     if (lane == 0) mbar_arrive(&empty[st]);
   }
 
-  if (!scores_fin) report_status(kDevRange, 43);
-  // partial results of this warp (its own split): rows < g
+  if (!q_fin) report_status(kDevRange, 42);
+  // An fp16 key operand that overflowed (|x| >= 65520 rounds to inf) or a NaN key makes a score
+  // inf or NaN (the padding query rows are zero: 0 * inf = NaN), which leaves the running max
+  // at +inf or the running sum NaN: one test of the final state covers every key of the split.
+  if (!(m_r < INFINITY) || !(l_r == l_r) || !(l_r < INFINITY)) report_status(kDevRange, 43);
   l_r += __shfl_xor_sync(0xffffffffu, l_r, 1);
   l_r += __shfl_xor_sync(0xffffffffu, l_r, 2);
-  const long long split = static_cast<long long>(bz) * a.parts_stride + static_cast<long long>(blockIdx.x) * 2 + nt;
+  // The two warps of a kv head each hold the softmax state of their half of every stage; warp
+  // nt = 1 hands its state to warp nt = 0 through shared memory (a named barrier per pair, 64
+  // threads), which merges the two and writes one partial per split, halving what the combine
+  // reads. Lane l of both warps holds the same rows and dimensions, so the merge is lane-wise.
+  float* xo = reinterpret_cast<float*>(xch) + hl * (32 * (4 * MT + 2));
+  if (nt == 1) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) xo[(4 * mt + e) * 32 + lane] = o[mt][e];
+    xo[(4 * MT) * 32 + lane] = m_r;
+    xo[(4 * MT + 1) * 32 + lane] = l_r;
+    asm volatile("bar.arrive %0, 64;" ::"r"(1 + hl) : "memory");
+    return;
+  }
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + hl) : "memory");
+  {
+    const float m1 = xo[(4 * MT) * 32 + lane], l1 = xo[(4 * MT + 1) * 32 + lane];
+    const float M = fmaxf(m_r, m1);
+    const float ref = (M == -INFINITY) ? 0.f : M;
+    const float a0 = fast_exp2(m_r - ref), a1 = fast_exp2(m1 - ref);
+    l_r = l_r * a0 + l1 * a1;
+    m_r = M;
+    // O^T columns are query rows 2t4 and 2t4 + 1: their factors sit on lanes 8t4 and 8t4 + 4
+    const float f00 = __shfl_sync(0xffffffffu, a0, 8 * t4), f01 = __shfl_sync(0xffffffffu, a0, 8 * t4 + 4);
+    const float f10 = __shfl_sync(0xffffffffu, a1, 8 * t4), f11 = __shfl_sync(0xffffffffu, a1, 8 * t4 + 4);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      o[mt][0] = o[mt][0] * f00 + xo[(4 * mt + 0) * 32 + lane] * f10;
+      o[mt][1] = o[mt][1] * f01 + xo[(4 * mt + 1) * 32 + lane] * f11;
+      o[mt][2] = o[mt][2] * f00 + xo[(4 * mt + 2) * 32 + lane] * f10;
+      o[mt][3] = o[mt][3] * f01 + xo[(4 * mt + 3) * 32 + lane] * f11;
+    }
+  }
+  // the merged partial of this split: rows < g
+  const long long split = static_cast<long long>(bz) * a.parts_stride + blockIdx.x;
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int row = 2 * t4 + e;
@@ -408,7 +472,8 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
 
 template <int D>
 constexpr int decode_smem_bytes() {
-  return 2 * dec::NST * dec::HPC * (D / 64) * dec::KB * 128 + dec::NST * dec::KB * (D / 2 * 8 + 64) + 3 * dec::NST * 8;
+  return 2 * dec::NST * dec::HPC * (D / 64) * dec::KB * 128 + dec::NST * dec::KB * (D / 2 * 8 + 64) + 3 * dec::NST * 8 +
+         dec::HPC * 32 * (4 * (D / 16) + 2) * 4;  // the warp pairs' exchange area
 }
 
 template <int D>
@@ -417,27 +482,32 @@ constexpr int decode_threads() {
 }
 
 // Log-sum-exp merge of the split partials. CTA (h, dq) merges query head h for the 32
-// dimensions 32dq .. 32dq+31, so D/32 CTAs share a head and the grid spreads over the SMs
-// (the merge reads every partial once and is latency-bound, not bandwidth-bound). The
-// global max comes from a block reduction over the partial maxima; then each warp sums a
-// strided share of the partials, one lane per dimension, and shared memory adds the warps.
+// dimensions 32dq .. 32dq+31, so D/32 CTAs share a head and the grid spreads over the SMs.
+// The merge is latency-bound (it reads each partial once), so each warp issues the loads of NB
+// of its splits at once and merges them online (running max, rescaled sum); one shared memory
+// step then merges the warps. NB is the smallest of 2, 4, 8, 16 that covers a warp's share in
+// one batch: a large NB costs registers (98 at NB = 16, two CTAs per SM), which a batched launch
+// of many CTAs pays in waves, while a few CTAs over many splits want every load in flight.
 constexpr int COMBINE_WARPS = 8;
 
 // Batched (grid.z = sequence, seq_lens non-null): sequence b's partials start at row
-// b * parts_stride, and only the 2 * ceil(seq_lens[b] / split_len) of its splits that hold keys
+// b * parts_stride, and only the ceil(seq_lens[b] / split_len) of its splits that hold keys
 // were written; out / lse advance by hq rows per sequence.
-template <int D>
-__global__ void __launch_bounds__(32 * COMBINE_WARPS) decode_combine_kernel(
+template <int D, int NB>
+__global__ void __launch_bounds__(32 * COMBINE_WARPS, NB <= 2 ? 8 : 1) decode_combine_kernel(
     const float* __restrict__ part_o, const float* __restrict__ part_ml, int n_split, int hq,
     __nv_bfloat16* __restrict__ out, float* __restrict__ lse, const int* __restrict__ seq_lens, int split_len,
-    int parts_stride) {
+    int parts_stride, int max_len) {
   __shared__ float red_acc[COMBINE_WARPS][32];
   __shared__ float red_l[COMBINE_WARPS];
-  __shared__ float warp_max[COMBINE_WARPS];
+  __shared__ float red_m[COMBINE_WARPS];
   pdl_wait();  // the partials of the previous kernel are complete and visible
   const int b = blockIdx.z;
   if (seq_lens) {
-    n_split = 2 * ((seq_lens[b] + split_len - 1) / split_len);
+    const int Lb = seq_lens[b];
+    // a length out of range had no partials written (the partial kernel reported it): merging
+    // nothing gives 0 / 0, NaN, as this sequence's output
+    n_split = (Lb >= 1 && Lb <= max_len) ? (Lb + split_len - 1) / split_len : 0;
     part_o += static_cast<long long>(b) * parts_stride * hq * D;
     part_ml += static_cast<long long>(b) * parts_stride * hq * 2;
     out += static_cast<long long>(b) * hq * D;
@@ -445,40 +515,51 @@ __global__ void __launch_bounds__(32 * COMBINE_WARPS) decode_combine_kernel(
   }
   const int h = blockIdx.x, d = 32 * blockIdx.y + (threadIdx.x & 31);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  // global max of the partial maxima
-  float M = -INFINITY;
-  for (int s = threadIdx.x; s < n_split; s += 32 * COMBINE_WARPS)
-    M = fmaxf(M, part_ml[(static_cast<long long>(s) * hq + h) * 2]);
+  float m = -INFINITY, acc = 0.f, l = 0.f;  // this lane's running merge (log2 domain max)
+  for (int s0 = warp; s0 < n_split; s0 += COMBINE_WARPS * NB) {
+    float2 ml[NB];
+    float ov[NB];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if (lane == 0) warp_max[warp] = M;
-  __syncthreads();
-  M = -INFINITY;
+    for (int u = 0; u < NB; ++u) {
+      const int sp = s0 + COMBINE_WARPS * u;
+      ml[u] = make_float2(-INFINITY, 0.f);
+      ov[u] = 0.f;
+      if (sp < n_split) {
+        const long long row = static_cast<long long>(sp) * hq + h;
+        ml[u] = *reinterpret_cast<const float2*>(part_ml + row * 2);
+        ov[u] = part_o[row * D + d];
+      }
+    }
 #pragma unroll
-  for (int w = 0; w < COMBINE_WARPS; ++w) M = fmaxf(M, warp_max[w]);
-  const float ref = (M == -INFINITY) ? 0.f : M;
-  // this warp's share of the partials
-  float acc = 0.f, lsum = 0.f;
-#pragma unroll 4
-  for (int s = warp; s < n_split; s += COMBINE_WARPS) {
-    const long long row = static_cast<long long>(s) * hq + h;
-    const float2 ml = *reinterpret_cast<const float2*>(part_ml + row * 2);
-    const float w = fast_exp2(ml.x - ref);
-    lsum += w * ml.y;
-    acc += w * part_o[row * D + d];
+    for (int u = 0; u < NB; ++u) {
+      const float M = fmaxf(m, ml[u].x);
+      const float ref = (M == -INFINITY) ? 0.f : M;
+      const float c = fast_exp2(m - ref), w = fast_exp2(ml[u].x - ref);
+      acc = acc * c + ov[u] * w;
+      l = l * c + ml[u].y * w;
+      m = M;
+    }
   }
   red_acc[warp][lane] = acc;
-  if (lane == 0) red_l[warp] = lsum;
+  if (lane == 0) {
+    red_l[warp] = l;
+    red_m[warp] = m;
+  }
   __syncthreads();
   if (warp == 0) {
-    float a = 0.f, l = 0.f;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < COMBINE_WARPS; ++w) M = fmaxf(M, red_m[w]);
+    const float ref = (M == -INFINITY) ? 0.f : M;
+    float sa = 0.f, sl = 0.f;
 #pragma unroll
     for (int w = 0; w < COMBINE_WARPS; ++w) {
-      a += red_acc[w][lane];
-      l += red_l[w];
+      const float c = fast_exp2(red_m[w] - ref);
+      sa += red_acc[w][lane] * c;
+      sl += red_l[w] * c;
     }
-    out[h * D + d] = __float2bfloat16(a / l);
-    if (lse && blockIdx.y == 0 && lane == 0) lse[h] = (M + __log2f(l)) * 0.69314718055994530942f;
+    out[h * D + d] = __float2bfloat16(sa / sl);
+    if (lse && blockIdx.y == 0 && lane == 0) lse[h] = (M + __log2f(sl)) * 0.69314718055994530942f;
   }
 }
 
@@ -493,20 +574,31 @@ struct AppendArgs {
   // batched paged form (grid.y = sequence): position seq_lens[b] - 1, pool row via the block table
   const int* seq_lens;
   const int* block_table;
-  int max_pages, page_size;
+  int max_pages, page_size, pool_pages, max_len;
 };
 
 template <int D>
 __global__ void decode_append_kernel(const __grid_constant__ AppendArgs a) {
   constexpr int P = D / 2;
   pdl_launch_dependents();  // the partial kernel may start; only its stage holding row p waits for us
+  pdl_wait();               // launched early itself: the kernel before it (which may produce k_new) is done
   const int h = blockIdx.x, lane = threadIdx.x, b = blockIdx.y;
   const bool paged = a.seq_lens != nullptr;
-  const int p = paged ? a.seq_lens[b] - 1 : a.p;  // logical position of the new token
-  const long long row =
-      paged ? static_cast<long long>(a.block_table[static_cast<long long>(b) * a.max_pages + p / a.page_size]) *
-                      a.page_size + p % a.page_size
-            : p;
+  int p = a.p;  // logical position of the new token
+  long long row = p;
+  if (paged) {
+    p = a.seq_lens[b] - 1;
+    if (p < 0 || p >= a.max_len) {  // a length out of range: append nothing
+      if (lane == 0) report_status(kDevIndex, 50);
+      return;
+    }
+    const int pg = a.block_table[static_cast<long long>(b) * a.max_pages + p / a.page_size];
+    if (pg < 0 || pg >= a.pool_pages) {  // a page outside the pool: write nothing
+      if (lane == 0) report_status(kDevIndex, 51);
+      return;
+    }
+    row = static_cast<long long>(pg) * a.page_size + p % a.page_size;
+  }
   const __nv_bfloat16* kr = a.k_new + (static_cast<long long>(b) * a.hkv + h) * D;
   __nv_bfloat16* kd = a.kcache + (row * a.hkv + h) * D;
   for (int pr = lane; pr < P; pr += 32) {

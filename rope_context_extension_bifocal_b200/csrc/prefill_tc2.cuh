@@ -128,6 +128,7 @@ struct Tc2Args {
   int q_off, Lq;
   float scale_log2;
   RopeSrc src;  // angles of the fused loads (FUSED only)
+  int test_skip_fill;  // test only (bifocal_test_set_fault): 1 + the fill CTA 0's producer never issues; 0 = off
   // A batch of chunks over a paged cache (FUSED only, nseq > 0). Launch-order entry s is the
   // chunk of sequence seq_id[s] (its block-table row): cached length seq_P0[s], chunk length
   // seq_C[s], factor seq_G[s], first row seq_qrow[s] of the packed q / out / lse rows (total_rows
@@ -137,6 +138,7 @@ struct Tc2Args {
   int nseq, total_rows;
   const int* block_table;
   int max_pages, page_size, seg_rows;
+  int pool_pages;  // a block-table entry outside [0, pool_pages) is reported and its segment read as zeros
   int tile_start[tc2::kMaxSeqs + 1];
   int seq_id[tc2::kMaxSeqs], seq_P0[tc2::kMaxSeqs], seq_C[tc2::kMaxSeqs], seq_G[tc2::kMaxSeqs],
       seq_qrow[tc2::kMaxSeqs];
@@ -279,8 +281,7 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
           prefetch_tensormap(&a.ql_map);
           prefetch_tensormap(&a.kl_map);
         }
-        int skip = -1;  // test only: never issue this fill (a volatile read inside the branch)
-        if (blockIdx.x == 0) skip = *reinterpret_cast<volatile int*>(&g_skip_fill_prefill);
+        const int skip = blockIdx.x == 0 ? a.test_skip_fill - 1 : -1;  // test only: never issue this fill
         uint32_t used = 0, par = 0;    // unfused ring: per slot, has a fill been issued, parity of the fills
         uint32_t kused = 0, kpar = 0;  // fused K ring (raw landed barriers)
         uint32_t vused = 0, vpar = 0;  // fused V ring
@@ -341,9 +342,11 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
             mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nvalid * a.seg_rows) * 256u);
             for (int sg = 0; sg < nvalid; ++sg) {
               const int j = t * BN + sg * a.seg_rows;
-              const int row =
-                  a.block_table[static_cast<long long>(b) * a.max_pages + j / a.page_size] * a.page_size +
-                  j % a.page_size;
+              const int pg = a.block_table[static_cast<long long>(b) * a.max_pages + j / a.page_size];
+              const bool pg_ok = pg >= 0 && pg < a.pool_pages;
+              if (!pg_ok) report_status(kDevIndex, 55);
+              // a bad entry loads the box that starts just past the pool's last row: TMA fills it with zeros
+              const int row = pg_ok ? pg * a.page_size + j % a.page_size : a.pool_pages * a.page_size;
               uint8_t* d0 = dst + sg * a.seg_rows * 128;
               tma_load_4d(d0, m, bar, 0, kvh, row, 0);
               tma_load_4d(d0 + HALF_BYTES, m, bar, 64, kvh, row, 0);
@@ -393,17 +396,18 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
         }
         // drain: every copy issued must have landed before the CTA may exit: the last fill of
         // every slot (the ones before it were consumed, or a later fill could not have been
-        // issued) and the last Q load
+        // issued) and the last Q load; the waits sleep between polls, so they take no issue
+        // slots from the warps still working
         if (FUSED) {
           for (int sl = 0; sl < NK3; ++sl)
-            if (kused & (1u << sl)) mbar_wait(&kraw[sl], ((kpar >> sl) & 1u) ^ 1u, 11);
+            if (kused & (1u << sl)) mbar_wait_sleepy(&kraw[sl], ((kpar >> sl) & 1u) ^ 1u, 11);
           for (int sl = 0; sl < NV2; ++sl)
-            if (vused & (1u << sl)) mbar_wait(&vfull[sl], ((vpar >> sl) & 1u) ^ 1u, 11);
-          mbar_wait(&q_raw, (q_loads - 1) & 1, 13);
+            if (vused & (1u << sl)) mbar_wait_sleepy(&vfull[sl], ((vpar >> sl) & 1u) ^ 1u, 11);
+          mbar_wait_sleepy(&q_raw, (q_loads - 1) & 1, 13);
         } else {
           for (int sl = 0; sl < NSLOT2; ++sl)
-            if (used & (1u << sl)) mbar_wait(&full[sl], ((par >> sl) & 1u) ^ 1u, 11);
-          mbar_wait(&q_full, (q_loads - 1) & 1, 13);
+            if (used & (1u << sl)) mbar_wait_sleepy(&full[sl], ((par >> sl) & 1u) ^ 1u, 11);
+          mbar_wait_sleepy(&q_full, (q_loads - 1) & 1, 13);
         }
       }
     } else if (FUSED && warp >= 10) {

@@ -62,7 +62,7 @@ struct PrepassArgs {
   // page_size + p % page_size.
   int nseq;
   const int* block_table;
-  int max_pages, page_size;
+  int max_pages, page_size, pool_pages;  // an entry outside [0, pool_pages) is reported, its row skipped
   int seq_id[64], seq_P0[64], seq_C[64], seq_qrow[64];
 };
 
@@ -128,8 +128,12 @@ __global__ void __launch_bounds__(256) rope_prepass_kernel(const __grid_constant
     int sq = 0;
     while (sq + 1 < a.nseq && a.seq_qrow[sq + 1] <= r_in) ++sq;
     p = a.seq_P0[sq] + (r_in - a.seq_qrow[sq]);
-    crow = static_cast<long long>(a.block_table[static_cast<long long>(a.seq_id[sq]) * a.max_pages + p / a.page_size]) *
-               a.page_size + p % a.page_size;
+    const int pg = a.block_table[static_cast<long long>(a.seq_id[sq]) * a.max_pages + p / a.page_size];
+    if (pg < 0 || pg >= a.pool_pages) {  // the table lies: write nothing for this row
+      if (lane == 0) report_status(kDevIndex, 54);
+      return;
+    }
+    crow = static_cast<long long>(pg) * a.page_size + p % a.page_size;
   }
   const int grp = lane >> 3, l8 = lane & 7;
   if (l8 >= LANES_PER_ROW) return;

@@ -43,11 +43,11 @@ def _clean_status():
     bfl.last_device_error()
 
 
-def small_prefill(scale_q=1.0, seed=71):
+def small_prefill(scale_q=1.0, seed=71, flags=0):
     L, hq, hkv, D, w0, wp = 1000, 4, 2, 128, 100, 256  # D 128, even GQA group: the ping-pong kernel
     q, k, v = si.random_qkv(seed, 1, L, hq, hkv, D, "bf16")
     q = (q.float() * scale_q).to(torch.bfloat16)
-    kw = dict(w0=w0, w_pretrained=wp, theta=1e4, mode=si.FREQ_INTERP)
+    kw = dict(w0=w0, w_pretrained=wp, theta=1e4, mode=si.FREQ_INTERP, flags=flags)
     out, lse, _, _ = bfl.bifocal_prefill(q.cuda(), k.cuda(), v.cuda(), **kw)
     return (q, k, v, kw), out, lse
 
@@ -58,17 +58,20 @@ def check_prefill_parity(case, out, lse):
     assert_close(out.cpu().float().numpy(), lse.cpu().numpy(), ro, rl, "prefill after a fault")
 
 
+@pytest.mark.parametrize("flags", [0, bfl.FLAG_FUSED_ROPE], ids=["rope_pass", "fused_loads"])
 @pytest.mark.parametrize("fill", [0, 1, 5])
-def test_prefill_skipped_fill_times_out_then_recovers(fill):
+def test_prefill_skipped_fill_times_out_then_recovers(fill, flags):
+    # the fused form's copies are issued by a transform warp between its tiles: a missing K fill
+    # leaves the transform warps waiting, a missing V fill the MMA issuer
     bfl.test_set_fault(bfl.FAULT_PREFILL_SKIP_FILL, fill, LIMIT_NS)
-    small_prefill()
+    small_prefill(flags=flags)
     word = bfl.device_status_word()
     assert word & 0xff == 1, hex(word)  # a bounded wait expired
     assert (word >> 8) in PREFILL_SITES, hex(word)
     assert bfl.last_device_error() == bfl.STATUS_TIMEOUT
     assert bfl.last_device_error() == 0  # reading cleared it
     bfl.test_set_fault()
-    case, out, lse = small_prefill()
+    case, out, lse = small_prefill(flags=flags)
     torch.cuda.synchronize()
     assert bfl.last_device_error() == 0
     check_prefill_parity(case, out, lse)
@@ -143,7 +146,11 @@ def test_decode_fp16_range_is_reported_then_recovers():
 
 def test_decode_cached_key_out_of_range_is_reported():
     q, kn, vn, kc, vc, L = decode_case()
-    kc[17, 1, 5] = 1e6  # a cached key no fp16 operand can hold, before or after its rotation
+    # a cached key no fp16 operand can hold, before or after its rotation, planted with both signs:
+    # negating a key negates its score, so one of the two rows scores +inf or NaN for every query
+    # head (a score of -inf alone would only give that key weight 0)
+    kc[17, 1, 5] = 1e6
+    kc[18, 1, 5] = -1e6
     run_decode((q, kn, vn, kc, vc, L))
     word = bfl.device_status_word()
     assert word & 0xff == 2 and (word >> 8) == 43, hex(word)
