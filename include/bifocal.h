@@ -281,7 +281,7 @@ BF_API bf_status_t bifocal_decode_paged(const void* q, const void* k_new, const 
  * device). There is no counterpart in the paper; this is a deployment convenience.
  * The split-KV partials live in a static device array of BIFOCAL_NOALLOC_SCRATCH_BYTES
  * (16 MiB) that every GPU loading the library holds until the process exits. A call needs
- * bifocal_decode_workspace_size(L, p) bytes of it (10.7 MB for 32 query heads of 128);
+ * bifocal_decode_workspace_size(L, p) bytes of it (5.3 MB for 32 query heads of 128);
  * larger problems are rejected with BF_ERR_WORKSPACE before any launch.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  * with that device current; make that first call before any stream capture. The address is

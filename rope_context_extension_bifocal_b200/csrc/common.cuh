@@ -110,6 +110,15 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+// bf16x2 -> packed fp32 pair (a bf16 is the upper half of its fp32); packed pair -> fp16x2 (RN)
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t f2_to_f16x2(uint64_t v) {
+  float lo, hi;
+  f2_unpack(v, lo, hi);
+  return pack_f16x2(lo, hi);
+}
 
 // ---------------------------------------------------------------------------------
 // Legacy warp-level tensor core path (used where tensor throughput is not the limit).

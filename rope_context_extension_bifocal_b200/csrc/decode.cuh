@@ -64,6 +64,17 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
 // TEST = true is the instantiation launched only while bifocal_test_set_fault has armed a
 // skipped stage: its producer stops issuing at that stage in CTA 0. The normal instantiation has
 // no trace of it (a changed loop bound in the producer cost up to 20 us per step).
+// Correction rotation of two pairs held as bf16x2 (x = elements d, d+1; y = elements d+P,
+// d+P+1) by {cos d, cos d+1, sin d, sin d+1}, on packed fp32 pairs; the result as fp16x2.
+__device__ __forceinline__ uint32_t rot_x(uint32_t x, uint32_t y, float4 cs) {
+  const uint64_t X = bf16x2_to_f2(x), Y = bf16x2_to_f2(y);
+  return f2_to_f16x2(f2_sub(f2_mul(X, f2_pack(cs.x, cs.y)), f2_mul(Y, f2_pack(cs.z, cs.w))));
+}
+__device__ __forceinline__ uint32_t rot_y(uint32_t x, uint32_t y, float4 cs) {
+  const uint64_t X = bf16x2_to_f2(x), Y = bf16x2_to_f2(y);
+  return f2_to_f16x2(f2_fma(X, f2_pack(cs.z, cs.w), f2_mul(Y, f2_pack(cs.x, cs.y))));
+}
+
 template <int D, bool TEST>
 __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_kernel(const __grid_constant__ DecodeArgs a) {
   using namespace dec;
@@ -185,17 +196,20 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
   }
   if (warp > 2 * HPC) {
     // ---------------- table warps (two, alternating stages): correction cos/sin per (key, pair).
-    // Each lane runs 4 chains (pairs lane and lane + 32, keys 0-7 and 8-15 of the stage): an
+    // Each lane runs 4 chains (pairs 2 lane and 2 lane + 1, keys 0-7 and 8-15 of the stage): an
     // exact angle at the chain's first key, then per-key steps: frequency interpolation adds
-    // omega_corr; position aliasing adds -omega unless the next key starts a group of G.
+    // omega_corr; position aliasing adds -omega unless the next key starts a group of G. A key
+    // row holds, per two pairs d, d + 1 (d even), {cos d, cos d+1, sin d, sin d+1}: the consumers'
+    // packed fp32 pairs.
     const int cw = warp - 2 * HPC - 1;  // 0 or 1
+    const bool lane_on = 2 * lane < P;
     float fi_c[2], fi_s[2], pa_c[2], pa_s[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const int pr = lane + 32 * e;
+      const int pr = 2 * lane + e;
       fi_c[e] = pa_c[e] = 1.f;
       fi_s[e] = pa_s[e] = 0.f;
-      if (pr < P) {
+      if (lane_on) {
         angle_cos_sin(omega_corr(pr), fi_c[e], fi_s[e]);
         angle_cos_sin(-a.omega[pr], pa_c[e], pa_s[e]);
       }
@@ -205,34 +219,36 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
       if (s >= NST && !__all_sync(0xffffffffu, mbar_wait_abortable(&empty[st], ((s / NST) - 1) & 1, 3, &s_abort)))
         break;
       const int j0 = jbeg + s * KB;
-      if (j0 < local_from) {  // some key of this stage is long-range
+      if (j0 < local_from && lane_on) {  // some key of this stage is long-range
         uint8_t* cs = sCS + st * STAGE_CS;
+        float c[2][2], sn[2][2];  // [pair 2 lane + e][chain hk]
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int pr = lane + 32 * e;
-          if (pr >= P) continue;
-          float c[2], sn[2];
+        for (int e = 0; e < 2; ++e)
 #pragma unroll
           for (int hk = 0; hk < 2; ++hk) {
+            const int pr = 2 * lane + e;
             const int jc = j0 + 8 * hk;
             const double ang0 = (a.mode == 0) ? static_cast<double>(jc) * omega_corr(pr)
                                               : static_cast<double>(jc / G - jc) * a.omega[pr];
-            angle_cos_sin(ang0, c[hk], sn[hk]);
+            angle_cos_sin(ang0, c[e][hk], sn[e][hk]);
           }
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
-            for (int hk = 0; hk < 2; ++hk) {
-              *reinterpret_cast<float2*>(cs + (8 * hk + kk) * CS_STRIDE + pr * 8) = make_float2(c[hk], sn[hk]);
+          for (int hk = 0; hk < 2; ++hk) {
+            *reinterpret_cast<float4*>(cs + (8 * hk + kk) * CS_STRIDE + lane * 16) =
+                make_float4(c[0][hk], c[1][hk], sn[0][hk], sn[1][hk]);
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
               float dc = fi_c[e], ds = fi_s[e];
               if (a.mode != 0) {
                 const bool stay = ((j0 + 8 * hk + kk + 1) % G) == 0;
                 dc = stay ? 1.f : pa_c[e];
                 ds = stay ? 0.f : pa_s[e];
               }
-              const float nc = c[hk] * dc - sn[hk] * ds;
-              sn[hk] = sn[hk] * dc + c[hk] * ds;
-              c[hk] = nc;
+              const float nc = c[e][hk] * dc - sn[e][hk] * ds;
+              sn[e][hk] = sn[e][hk] * dc + c[e][hk] * ds;
+              c[e][hk] = nc;
             }
           }
         }
@@ -329,15 +345,12 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
         mma_f16_16816(so, a1, bf16x2_to_f16x2(r[2]), bf16x2_to_f16x2(r[3]));
       }
       if (tile_long) {
+        // {cos d, cos d+1, sin d, sin d+1} of pairs d = 16kc + 2t4 (and d + 8), this lane's key
         const float4 c01 = *reinterpret_cast<const float4*>(cs + key_mine * CS_STRIDE + (16 * kc + 2 * t4) * 8);
         const float4 c89 = *reinterpret_cast<const float4*>(cs + key_mine * CS_STRIDE + (16 * kc + 8 + 2 * t4) * 8);
-        const float2 x0 = unpack_bf16x2(r[0]), x1 = unpack_bf16x2(r[1]);
-        const float2 y0 = unpack_bf16x2(r[2]), y1 = unpack_bf16x2(r[3]);
-        // pair (x, y) -> (x c - y s, y c + x s)
-        const uint32_t rx0 = pack_f16x2(x0.x * c01.x - y0.x * c01.y, x0.y * c01.z - y0.y * c01.w);
-        const uint32_t ry0 = pack_f16x2(y0.x * c01.x + x0.x * c01.y, y0.y * c01.z + x0.y * c01.w);
-        const uint32_t rx1 = pack_f16x2(x1.x * c89.x - y1.x * c89.y, x1.y * c89.z - y1.y * c89.w);
-        const uint32_t ry1 = pack_f16x2(y1.x * c89.x + x1.x * c89.y, y1.y * c89.z + x1.y * c89.w);
+        // pair (x, y) -> (x c - y s, y c + x s), two pairs per packed fp32 instruction
+        const uint32_t rx0 = rot_x(r[0], r[2], c01), ry0 = rot_y(r[0], r[2], c01);
+        const uint32_t rx1 = rot_x(r[1], r[3], c89), ry1 = rot_y(r[1], r[3], c89);
         uint32_t a0[4] = {qa_l[kc][0], 0u, qa_l[kc][1], 0u};
         uint32_t a1[4] = {qa_l[kc + KCP][0], 0u, qa_l[kc + KCP][1], 0u};
         mma_f16_16816(sl, a0, rx0, rx1);

@@ -123,12 +123,6 @@ __device__ __forceinline__ void st_shared16(uint32_t addr, const uint4& v) {
 }
 
 // Two bf16 of one word as a packed pair of fp32 (a bf16 is the high half of its fp32).
-__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) { return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)); }
-__device__ __forceinline__ uint32_t f2_to_f16x2(uint64_t v) {
-  float lo, hi;
-  f2_unpack(v, lo, hi);
-  return pack_f16x2(lo, hi);
-}
 
 // 8 pairs: x = elements 8c..8c+7 (bf16, in a), y = their partners 64 later (bf16, in b).
 // (x, y) -> (x cos - y sin, y cos + x sin), rounded to fp16, written back over a and b.
