@@ -154,6 +154,10 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
   using namespace tc2;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ uint64_t full[NSLOT2], empty[NSLOT2], s_full[2], p_ready[2], o_done[2], q_full, q_free, mma_drain;
+  // P is handed over in two halves (keys 0-63, 64-127 of the tile): p_lo releases the first
+  // half's P.V while the softmax finishes the second; o_lo completes when that half's P.V has
+  // run (waited on only when the second half needs a new row reference after the first was sent)
+  __shared__ uint64_t p_lo[2], o_lo[2];
   // fused rings: K raw landed / K operand ready / K slot free; V landed / V slot free; raw Q landed
   __shared__ uint64_t kraw[NK3], kfull[NK3], kempty[NK3], vfull[NV2], vempty[NV2], q_raw, v_fix[2];
   __shared__ uint32_t tmem_base_sh;
@@ -229,7 +233,9 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_ready[i], 4);
+      mbar_init(&p_lo[i], 4);
       mbar_init(&o_done[i], 1);
+      mbar_init(&o_lo[i], 1);
     }
     mbar_init(&q_raw, 1);
     mbar_init(&v_fix[0], rl::NXF);  // one per visit of a tile past a paged sequence's end (at most two:
@@ -487,15 +493,18 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
           }
           mma_commit(&s_full[x]);
         };
-        auto pv = [&](int x, int v) {
+        // O_x += P_x(v) V(v) over keys 64h .. 64h + 63 (four 16-key steps); h = 0 commits o_lo, h = 1 o_done
+        auto pv_half = [&](int x, int v, int h) {
           const uint64_t b0 = dv0 + static_cast<uint64_t>(v_slot(v) * (SLOT_BYTES >> 4));
           const uint32_t p_col = tmem + (x == 0 ? COL_SA : COL_SB);
           const uint32_t o_col = tmem + (x == 0 ? COL_OA : COL_OB);
           const uint32_t acc0 = v > 0;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kk = 4 * h + k4;
             mma_ts(o_col, p_col + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), IDESC_PV, kk > 0 ? 1u : acc0);
-          mma_commit(&o_done[x]);
+          }
+          mma_commit(h == 0 ? &o_lo[x] : &o_done[x]);
         };
         // visit 0: S_A, S_B
         if (ok) ok = mbar_wait_abortable(k_full(0), k_full_ph(0), 21, &s_abort);
@@ -507,8 +516,8 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
           if (reload_q && v_sw == 1) mma_commit(&q_free);
         }
         for (int v = 0; v < nv && ok; ++v) {
-          // O_A += P_A(v) V(v)
-          if (!mbar_wait_abortable(&p_ready[0], v & 1, 22, &s_abort) ||
+          // O_A += P_A(v) V(v), first half as soon as the softmax has sent it
+          if (!mbar_wait_abortable(&p_lo[0], v & 1, 22, &s_abort) ||
               !mbar_wait_abortable(v_full(v), v_full_ph(v), 23, &s_abort)) {
             ok = false;
             break;
@@ -522,7 +531,13 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
             }
           }
           fence_after();
-          pv(0, v);
+          pv_half(0, v, 0);
+          if (!mbar_wait_abortable(&p_ready[0], v & 1, 29, &s_abort)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          pv_half(0, v, 1);
           const bool more = v + 1 < nv;
           if (more) {
             if (reload_q && v + 1 == v_sw && !mbar_wait_abortable(&q_full, 1, 24, &s_abort)) {
@@ -537,12 +552,18 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
             qk(0, v + 1);  // S_A is free: PV_A(v) was issued before
           }
           // O_B += P_B(v) V(v)
-          if (!mbar_wait_abortable(&p_ready[1], v & 1, 26, &s_abort)) {
+          if (!mbar_wait_abortable(&p_lo[1], v & 1, 26, &s_abort)) {
             ok = false;
             break;
           }
           fence_after();
-          pv(1, v);
+          pv_half(1, v, 0);
+          if (!mbar_wait_abortable(&p_ready[1], v & 1, 33, &s_abort)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          pv_half(1, v, 1);
           mma_commit(v_empty(v));
           if (more) {
             qk(1, v + 1);
@@ -585,42 +606,111 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
       const int hi = (kind == ORIG_LOCAL) ? a.w0 : 0x7fffffff;  //      and i - j < hi
       float alpha = 1.f, rs = 0.f;
       bool grow = false;
-      uint32_t pk[64];  // P of the whole row, bf16 pairs; stored to TMEM once it is final
+      uint32_t pk[64];  // P of the whole row, bf16 pairs (keys 2u, 2u + 1 in pk[u])
       // Fast path (unmasked visits once the row has a reference): one pass with the current
-      // reference m_ref. m_ref never exceeds the running max, so every P term is bounded by
-      // 2^(running max - m_ref); the row sum bounds them all, and a sum above 2^24 (or not
-      // finite) sends the visit to the exact two-pass path below.
-      // Both choices below are made for the whole warp: each path reads S with tcgen05.ld,
-      // a warp-collective (.sync.aligned) instruction, so the lanes must not split between
-      // them. A row that needs the exact path (its reference is still -inf: no key of the
-      // earlier visits was in range, as happens in a sliding window; or its fast sum
-      // overflowed) takes the whole warp with it; the exact path is correct for every row.
+      // reference m_ref, half a row at a time. m_ref never exceeds the running max, so every P
+      // term is bounded by 2^(running max - m_ref); a half whose sum stays within 2^24 has no
+      // term that could overflow. The first half (keys 0-63) goes to the MMA as soon as it is
+      // known to be safe, so its P.V runs while the second half is computed. A first half above
+      // 2^24 (or not finite) sends the visit to the exact two-pass path below; a second half
+      // above it, after the first was sent, takes a new reference for the second half and
+      // rescales O once the first half's P.V has run (o_lo).
+      // Every choice is made for the whole warp: each path reads S with tcgen05.ld, a
+      // warp-collective (.sync.aligned) instruction, so the lanes must not split between them.
+      // A row that needs the exact path (its reference is still -inf: no key of the earlier
+      // visits was in range, as happens in a sliding window; or its fast sum overflowed) takes
+      // the whole warp with it; the exact path is correct for every row.
       bool exact = __any_sync(0xffffffffu, masked || m_ref == -INFINITY);
+      bool lo_sent = false;
       if (!exact) {
         // pairs of columns go through the packed f32x2 FMA and add
-        const uint64_t sc2 = f2_pack(sc, sc), nref2 = f2_pack(-m_ref, -m_ref);
-        uint64_t r4[4];
+        const uint64_t sc2 = f2_pack(sc, sc);
+        auto half_pass = [&](int c_lo, uint64_t nref2) -> float {
+          uint64_t r4[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) r4[u] = f2_pack(0.f, 0.f);
+          for (int u = 0; u < 4; ++u) r4[u] = f2_pack(0.f, 0.f);
 #pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          float s[32];
-          tmem_ld32(s_col + c0, s);
-          wait_ld();
+          for (int c0 = c_lo; c0 < c_lo + 64; c0 += 32) {
+            float s[32];
+            tmem_ld32(s_col + c0, s);
+            wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sc2, nref2), x0, x1);
-            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-            r4[(c >> 1) & 3] = f2_add(r4[(c >> 1) & 3], f2_pack(p0, p1));
-            pk[(c0 + c) >> 1] = pack_bf16x2(p0, p1);
+            for (int c = 0; c < 32; c += 2) {
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sc2, nref2), x0, x1);
+              const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+              r4[(c >> 1) & 3] = f2_add(r4[(c >> 1) & 3], f2_pack(p0, p1));
+              pk[(c0 + c) >> 1] = pack_bf16x2(p0, p1);
+            }
           }
-        }
-        float r8[8];
+          float r8[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) f2_unpack(r4[u], r8[2 * u], r8[2 * u + 1]);
-        rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
-        exact = __any_sync(0xffffffffu, !(rs <= 16777216.f));
+          for (int u = 0; u < 4; ++u) f2_unpack(r4[u], r8[2 * u], r8[2 * u + 1]);
+          return ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+        };
+        const float rs_lo = half_pass(0, f2_pack(-m_ref, -m_ref));
+        exact = __any_sync(0xffffffffu, !(rs_lo <= 16777216.f));
+        if (!exact) {
+          // send the first half: P over columns 0-31 of the S buffer (S of keys 0-63 is consumed)
+          tmem_st32(s_col, pk);
+          wait_st();
+          fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_lo[x]);
+          lo_sent = true;
+          float rs_hi = half_pass(64, f2_pack(-m_ref, -m_ref));
+          rs = rs_lo + rs_hi;
+          if (__any_sync(0xffffffffu, !(rs_hi <= 16777216.f))) {
+            // Rare: the second half's terms outgrow the reference the first half was sent with.
+            // Its S columns (64-127) are intact: take the raw max over them, move the reference
+            // where it grew past the threshold, and recompute the second half against it.
+            float m8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) m8[u] = -INFINITY;
+#pragma unroll
+            for (int c0 = 64; c0 < 128; c0 += 32) {
+              float s[32];
+              tmem_ld32(s_col + c0, s);
+              wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; c += 8)
+#pragma unroll
+                for (int u = 0; u < 8; ++u) m8[u] = fmaxf(m8[u], s[c + u]);
+            }
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
+                             sc;
+            if (mx > m_ref + RESCALE_THRESHOLD) {
+              alpha = fast_exp2(m_ref - mx);
+              grow = true;
+              m_ref = mx;
+            }
+            rs_hi = half_pass(64, f2_pack(-m_ref, -m_ref));
+            rs = rs_lo * alpha + rs_hi;  // l_sum * alpha + rs below: both earlier sums rescaled
+            // O must hold the first half's P.V (old reference) before it is rescaled, and the
+            // second half's P.V (new reference) must not start before: it waits for p_ready
+            if (!__all_sync(0xffffffffu, mbar_wait_abortable(&o_lo[x], v & 1, 34, &s_abort))) {
+              ok = false;
+              break;
+            }
+            fence_after();
+            if (__any_sync(0xffffffffu, grow)) {  // warp-uniform; rows that need none scale by 1
+              const float f = grow ? alpha : 1.f;
+#pragma unroll 1
+              for (int c0 = 0; c0 < 128; c0 += 32) {
+                float ov[32];
+                tmem_ld32(o_col + c0, ov);
+                wait_ld();
+                uint32_t ou[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) ou[u] = __float_as_uint(ov[u] * f);
+                tmem_st32(o_col + c0, ou);
+              }
+            }
+          }
+          l_sum = l_sum * alpha + rs;
+          tmem_st32(s_col + 32, pk + 32);  // the second half: columns 32-63
+        }
       }
       if (exact) {
         // pass 1: raw row max over the 128 columns
@@ -676,35 +766,38 @@ __global__ void __launch_bounds__(tc2::NTHREADS2, 1) attn_tc2_kernel(const __gri
           }
         }
         rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
-      }
-      l_sum = l_sum * alpha + rs;
-      tmem_st32(s_col, pk);       // P over the first 64 columns of the S buffer
-      tmem_st32(s_col + 32, pk + 32);
-      // O_x must hold PV(v-1) before it is rescaled and before PV(v) adds to it
-      if (v >= 1) {
-        if (!__all_sync(0xffffffffu, mbar_wait_abortable(&o_done[x], (v - 1) & 1, 31, &s_abort))) {
-          ok = false;
-          break;
-        }
-        fence_after();
-        if (__any_sync(0xffffffffu, grow)) {  // warp-uniform; rows that need none scale by 1
-          const float f = grow ? alpha : 1.f;
+        l_sum = l_sum * alpha + rs;
+        tmem_st32(s_col, pk);  // P over the first 64 columns of the S buffer
+        tmem_st32(s_col + 32, pk + 32);
+        // O_x must hold PV(v-1) before it is rescaled and before PV(v) adds to it
+        if (v >= 1) {
+          if (!__all_sync(0xffffffffu, mbar_wait_abortable(&o_done[x], (v - 1) & 1, 31, &s_abort))) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          if (__any_sync(0xffffffffu, grow)) {  // warp-uniform; rows that need none scale by 1
+            const float f = grow ? alpha : 1.f;
 #pragma unroll 1
-          for (int c0 = 0; c0 < 128; c0 += 32) {
-            float ov[32];
-            tmem_ld32(o_col + c0, ov);
-            wait_ld();
-            uint32_t ou[32];
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+              float ov[32];
+              tmem_ld32(o_col + c0, ov);
+              wait_ld();
+              uint32_t ou[32];
 #pragma unroll
-            for (int u = 0; u < 32; ++u) ou[u] = __float_as_uint(ov[u] * f);
-            tmem_st32(o_col + c0, ou);
+              for (int u = 0; u < 32; ++u) ou[u] = __float_as_uint(ov[u] * f);
+              tmem_st32(o_col + c0, ou);
+            }
           }
         }
       }
       wait_st();
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready[x]);
+      if (lane == 0) {
+        if (!lo_sent) mbar_arrive(&p_lo[x]);
+        mbar_arrive(&p_ready[x]);
+      }
     }
     // epilogue: O / l -> bf16, LSE
     if (ok && nv > 0 && __all_sync(0xffffffffu, mbar_wait_abortable(&o_done[x], (nv - 1) & 1, 32, &s_abort))) {

@@ -25,7 +25,7 @@ from tests.gpu_helpers import assert_close
 
 pytestmark = pytest.mark.gpu
 
-PREFILL_SITES = set(range(10, 33))  # the bounded waits of the ping-pong prefill kernel
+PREFILL_SITES = set(range(10, 35))  # the bounded waits of the ping-pong prefill kernel
 DECODE_SITES = {1, 2, 3, 4, 5}       # the bounded waits of the split-KV decode kernel
 LIMIT_NS = 50_000_000
 

@@ -61,7 +61,60 @@ class Bar:
         return (self.phase & 1) != parity
 
 
-def run_protocol(sch, rnd, skip_q_free_wait=False):
+def softmax_prog(x, nv, rnd):
+    """One softmax group's steps: per visit it waits for S, then sends P in two halves (p_lo, then
+    p_ready) by one of the kernel's three routes, chosen at random per visit:
+    - fast: both halves against the current reference, no wait on O;
+    - rare: the first half is sent, then the second half needs a new reference, so O is rescaled
+      once the first half's P.V has run (o_lo) and before the second half is sent;
+    - exact: both halves computed before either is sent; O is rescaled once the previous visit's
+      P.V has run (o_done).
+    After the last visit the epilogue waits for the last P.V."""
+    prog = []
+    for v in range(nv):
+        prog.append(("wait_s", x, v))
+        route = rnd.choice(("fast", "rare", "exact"))
+        if route == "fast":
+            prog += [("arrive_lo", x), ("arrive_hi", x)]
+        elif route == "rare":
+            prog += [("arrive_lo", x), ("wait_olo", x, v), ("rescale", x), ("arrive_hi", x)]
+        else:
+            if v >= 1:
+                prog += [("wait_o", x, v - 1), ("rescale", x)]
+            prog += [("arrive_lo", x), ("arrive_hi", x)]
+    if nv:
+        prog.append(("wait_o", x, nv - 1))
+    return prog
+
+
+def softmax_step(st, x, s_full, p_lo, p_ready, o_lo, o_done, pipe, skip_olo_wait=False):
+    """One softmax step of softmax_prog; False while it has to wait."""
+    if st[0] == "wait_s":
+        if not s_full[x].passed(st[2] & 1):
+            return False
+        assert s_full[x].phase == st[2] + 1, "S parity alias"
+    elif st[0] == "wait_o":
+        if not o_done[x].passed(st[2] & 1):
+            return False
+        assert o_done[x].phase >= st[2] + 1, "O parity alias"
+    elif st[0] == "wait_olo":
+        if skip_olo_wait:
+            return True
+        if not o_lo[x].passed(st[2] & 1):
+            return False
+        assert o_lo[x].phase == st[2] + 1, "o_lo parity alias"
+    elif st[0] == "rescale":
+        assert not any(e[0] in ("o_lo", "o_done") and e[1] == x for e in pipe), "O rescaled while a P.V into it runs"
+    elif st[0] == "arrive_lo":
+        for _ in range(4):
+            p_lo[x].arrive()
+    else:
+        for _ in range(4):
+            p_ready[x].arrive()
+    return True
+
+
+def run_protocol(sch, rnd, skip_q_free_wait=False, skip_olo_wait=False):
     nv = sch["n_long"] + sch["n_loc"]
     has_long, has_orig = sch["n_long"] > 0, sch["n_loc"] > 0
     reload_q = has_long and has_orig
@@ -69,6 +122,7 @@ def run_protocol(sch, rnd, skip_q_free_wait=False):
     full = [Bar(1) for _ in range(NSLOT)]
     empty = [Bar(1) for _ in range(NSLOT)]
     s_full, p_ready, o_done = [Bar(1), Bar(1)], [Bar(4), Bar(4)], [Bar(1), Bar(1)]
+    p_lo, o_lo = [Bar(4), Bar(4)], [Bar(1), Bar(1)]
     q_full, q_free = Bar(1), Bar(1)
     tma, pipe = [], []
     state = {"q_readers": 0}
@@ -87,31 +141,22 @@ def run_protocol(sch, rnd, skip_q_free_wait=False):
         mma.append(("commit", q_free))
     for v in range(nv):
         vs = (2 * v + 1) % NSLOT
-        mma += [("wait", p_ready[0], v & 1), ("wait", full[vs], ((2 * v + 1) // NSLOT) & 1), ("pv", 0)]
+        mma += [("wait", p_lo[0], v & 1), ("wait", full[vs], ((2 * v + 1) // NSLOT) & 1), ("pvlo", 0),
+                ("wait", p_ready[0], v & 1), ("pvhi", 0)]
         more = v + 1 < nv
         if more:
             if reload_q and v + 1 == v_sw:
                 mma.append(("wait", q_full, 1))
             k2 = (2 * (v + 1)) % NSLOT
             mma += [("wait", full[k2], ((2 * (v + 1)) // NSLOT) & 1), ("qk", 0)]
-        mma += [("wait", p_ready[1], v & 1), ("pv", 1), ("commit", empty[vs])]
+        mma += [("wait", p_lo[1], v & 1), ("pvlo", 1), ("wait", p_ready[1], v & 1), ("pvhi", 1),
+                ("commit", empty[vs])]
         if more:
             mma += [("qk", 1), ("commit", empty[(2 * (v + 1)) % NSLOT])]
             if reload_q and v + 2 == v_sw:
                 mma.append(("commit", q_free))
 
-    def softmax_prog(x):
-        prog = []
-        for v in range(nv):
-            prog.append(("wait_s", x, v))
-            if v >= 1:
-                prog.append(("wait_o", x, v - 1))
-            prog.append(("arrive", x))
-        if nv:
-            prog.append(("wait_o", x, nv - 1))
-        return prog
-
-    progs = {"prod": prod, "mma": mma, "smA": softmax_prog(0), "smB": softmax_prog(1)}
+    progs = {"prod": prod, "mma": mma, "smA": softmax_prog(0, nv, rnd), "smB": softmax_prog(1, nv, rnd)}
     pc = {k: 0 for k in progs}
 
     def step_prod():
@@ -141,7 +186,9 @@ def run_protocol(sch, rnd, skip_q_free_wait=False):
         if st[0] == "qk":
             state["q_readers"] += 1
             pipe.append(("s_full", st[1]))
-        elif st[0] == "pv":
+        elif st[0] == "pvlo":
+            pipe.append(("o_lo", st[1]))
+        elif st[0] == "pvhi":
             pipe.append(("o_done", st[1]))
         else:
             pipe.append(("bar", st[1]))
@@ -154,24 +201,14 @@ def run_protocol(sch, rnd, skip_q_free_wait=False):
             s_full[arg].arrive()
         elif kind == "o_done":
             o_done[arg].arrive()
+        elif kind == "o_lo":
+            o_lo[arg].arrive()
         else:
             arg.arrive()
         return True
 
     def step_softmax(name, x):
-        st = progs[name][pc[name]]
-        if st[0] == "wait_s":
-            if not s_full[x].passed(st[2] & 1):
-                return False
-            assert s_full[x].phase == st[2] + 1, "S parity alias"
-        elif st[0] == "wait_o":
-            if not o_done[x].passed(st[2] & 1):
-                return False
-            assert o_done[x].phase >= st[2] + 1, "O parity alias"
-        else:
-            for _ in range(4):
-                p_ready[x].arrive()
-        return True
+        return softmax_step(progs[name][pc[name]], x, s_full, p_lo, p_ready, o_lo, o_done, pipe, skip_olo_wait)
 
     def actors():
         out = []
@@ -242,7 +279,7 @@ def test_model_catches_a_missing_q_free_wait():
 NK3, NV2 = 3, 2  # fused form: K ring (raw tile lands, transform warps rotate it in place) and V ring
 
 
-def run_protocol_fused(sch, rnd, skip_kraw_wait=False):
+def run_protocol_fused(sch, rnd, skip_kraw_wait=False, skip_olo_wait=False):
     """The fused form's protocol: the TMA producer brings raw Q, raw K tiles (ring of three) and V
     tiles (ring of two); the transform warps rotate Q and each K tile in place once its raw bytes
     have landed; the MMA issuer, tensor pipe and softmax groups are those of the other form, with
@@ -258,6 +295,7 @@ def run_protocol_fused(sch, rnd, skip_kraw_wait=False):
     vfull = [Bar(1) for _ in range(NV2)]
     vempty = [Bar(1) for _ in range(NV2)]
     s_full, p_ready, o_done = [Bar(1), Bar(1)], [Bar(4), Bar(4)], [Bar(1), Bar(1)]
+    p_lo, o_lo = [Bar(4), Bar(4)], [Bar(1), Bar(1)]
     q_raw, q_full, q_free = Bar(1), Bar(1), Bar(1)
     tma, pipe = [], []
     state = {"q_readers": 0, "k_readers": [0] * NK3, "v_readers": [0] * NV2, "k_landed": [0] * NK3}
@@ -288,30 +326,21 @@ def run_protocol_fused(sch, rnd, skip_kraw_wait=False):
     if reload_q and v_sw == 1:
         mma.append(("commit", q_free))
     for v in range(nv):
-        mma += [("wait", p_ready[0], v & 1), ("wait", vfull[v % NV2], (v // NV2) & 1), ("pv", 0, v)]
+        mma += [("wait", p_lo[0], v & 1), ("wait", vfull[v % NV2], (v // NV2) & 1), ("pvlo", 0, v),
+                ("wait", p_ready[0], v & 1), ("pvhi", 0, v)]
         more = v + 1 < nv
         if more:
             if reload_q and v + 1 == v_sw:
                 mma.append(("wait", q_full, 1))
             mma += [("wait", kfull[(v + 1) % NK3], ((v + 1) // NK3) & 1), ("qk", 0, v + 1)]
-        mma += [("wait", p_ready[1], v & 1), ("pv", 1, v), ("commit", vempty[v % NV2])]
+        mma += [("wait", p_lo[1], v & 1), ("pvlo", 1, v), ("wait", p_ready[1], v & 1), ("pvhi", 1, v),
+                ("commit", vempty[v % NV2])]
         if more:
             mma += [("qk", 1, v + 1), ("commit", kempty[(v + 1) % NK3])]
             if reload_q and v + 2 == v_sw:
                 mma.append(("commit", q_free))
 
-    def softmax_prog(x):
-        prog = []
-        for v in range(nv):
-            prog.append(("wait_s", x, v))
-            if v >= 1:
-                prog.append(("wait_o", x, v - 1))
-            prog.append(("arrive", x))
-        if nv:
-            prog.append(("wait_o", x, nv - 1))
-        return prog
-
-    progs = {"prod": prod, "xf": xf, "mma": mma, "smA": softmax_prog(0), "smB": softmax_prog(1)}
+    progs = {"prod": prod, "xf": xf, "mma": mma, "smA": softmax_prog(0, nv, rnd), "smB": softmax_prog(1, nv, rnd)}
     pc = {k: 0 for k in progs}
 
     def land(kind, arg):
@@ -388,9 +417,9 @@ def run_protocol_fused(sch, rnd, skip_kraw_wait=False):
             state["q_readers"] += 1
             state["k_readers"][st[2] % NK3] += 1
             pipe.append(("s_full", st[1], st[2]))
-        elif st[0] == "pv":
+        elif st[0] in ("pvlo", "pvhi"):
             state["v_readers"][st[2] % NV2] += 1
-            pipe.append(("o_done", st[1], st[2]))
+            pipe.append(("o_lo" if st[0] == "pvlo" else "o_done", st[1], st[2]))
         else:
             pipe.append(("bar", st[1], None))
         return True
@@ -401,27 +430,15 @@ def run_protocol_fused(sch, rnd, skip_kraw_wait=False):
             state["q_readers"] -= 1
             state["k_readers"][v % NK3] -= 1
             s_full[arg].arrive()
-        elif kind == "o_done":
+        elif kind in ("o_lo", "o_done"):
             state["v_readers"][v % NV2] -= 1
-            o_done[arg].arrive()
+            (o_lo if kind == "o_lo" else o_done)[arg].arrive()
         else:
             arg.arrive()
         return True
 
     def step_softmax(name, x):
-        st = progs[name][pc[name]]
-        if st[0] == "wait_s":
-            if not s_full[x].passed(st[2] & 1):
-                return False
-            assert s_full[x].phase == st[2] + 1, "S parity alias"
-        elif st[0] == "wait_o":
-            if not o_done[x].passed(st[2] & 1):
-                return False
-            assert o_done[x].phase >= st[2] + 1, "O parity alias"
-        else:
-            for _ in range(4):
-                p_ready[x].arrive()
-        return True
+        return softmax_step(progs[name][pc[name]], x, s_full, p_lo, p_ready, o_lo, o_done, pipe, skip_olo_wait)
 
     def actors():
         out = []
@@ -471,6 +488,26 @@ def test_fused_model_catches_a_missing_raw_wait():
     for _ in range(100):
         try:
             run_protocol_fused(sch, rnd, skip_kraw_wait=True)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
+def test_model_catches_a_rescale_before_the_first_half_ran():
+    # planted mistake: the rare route rescales O without waiting for the first half's P.V
+    sch = schedule(2048, 17, 300, "bifocal")
+    rnd = random.Random(13)
+    caught = 0
+    for _ in range(200):
+        try:
+            run_protocol(sch, rnd, skip_olo_wait=True)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+    caught = 0
+    for _ in range(200):
+        try:
+            run_protocol_fused(sch, rnd, skip_olo_wait=True)
         except AssertionError:
             caught += 1
     assert caught > 0
