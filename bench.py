@@ -33,14 +33,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel,
-# from one single-pass ncu capture of a full-size launch, keyed by the SHA-256 of the kernel's
-# sources at capture time: when the sources no longer match, the kernel has changed since the
-# counters were taken and traffic is null.
+# from one single-pass ncu capture of a full-size launch (L = 131072, the bench workload), keyed
+# by the SHA-256 of the kernel's sources at capture time: when the sources no longer match, the
+# kernel has changed since the counters were taken and traffic is null.
 TRAFFIC = {
     "prefill_attention": {
-        "bytes_per_launch": 60.62e9 + 1.11e9,
-        "sources": ["common.cuh", "prefill_tc.cuh", "prefill_tc2.cuh"],
-        "sha256": "b5d7f2e31ad8806c5666de6ea4e04cfb217ab0415fab212aa6554ff7b5b692fb",
+        "bytes_per_launch": 4.99e9 + 1.07e9,
+        "sources": ["common.cuh", "prefill_tc.cuh", "prefill_tc2.cuh", "rope_loads.cuh"],
+        "sha256": "106d9b5065b65889cceba8fcd35e1efe2d8acb7fa1ffd87c2a35f5119e62651f",
     },
 }
 
