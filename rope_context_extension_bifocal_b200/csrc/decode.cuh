@@ -147,9 +147,14 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
                                                                                  : nstage;
       uint32_t used = 0, par = 0;  // per slot: has a fill been issued, parity of the fills issued
       // paged: the block-table entry of the current page and, loaded one page ahead, of the next
-      // (the stages of a split walk its pages in order, so the load has a page of stages to land)
-      int cur_idx = -1, cur_row0 = 0;
-      int nxt_pg = paged ? a.block_table[static_cast<long long>(bz) * a.max_pages + jbeg / a.page_size] : 0;
+      // (the stages of a split walk its pages in order, so the load has a page of stages to land).
+      // The page index and the offset in it advance by KB keys per stage without a division.
+      const int* trow = a.block_table + static_cast<long long>(bz) * a.max_pages;
+      int cur_idx = paged ? jbeg / a.page_size : 0;
+      int cur_off = paged ? jbeg - cur_idx * a.page_size : 0;
+      int cur_row0 = 0;
+      bool new_page = true;
+      int nxt_pg = paged ? trow[cur_idx] : 0;
       for (int s = 0; s < n_issue; ++s) {
         const int st = s % NST;
         if (s >= NST && !mbar_wait_abortable(&empty[st], ((s / NST) - 1) & 1, 1, &s_abort)) break;
@@ -160,17 +165,22 @@ __global__ void __launch_bounds__((2 * dec::HPC + 3) * 32, 1) decode_partial_ker
         // pool row of logical key j0 (pages hold a multiple of KB keys, so a stage is one page's)
         int row = j0;
         if (paged) {
-          const int idx = j0 / a.page_size;
-          if (idx != cur_idx) {
+          if (new_page) {
             const int pg = nxt_pg;
-            cur_idx = idx;
-            nxt_pg = idx + 1 < a.max_pages ? a.block_table[static_cast<long long>(bz) * a.max_pages + idx + 1] : 0;
+            nxt_pg = cur_idx + 1 < a.max_pages ? trow[cur_idx + 1] : 0;
             const bool pg_ok = pg >= 0 && pg < a.pool_pages;
             if (!pg_ok) report_status(kDevIndex, 53);
             // a bad entry loads stages that start just past the pool's last row: TMA fills them with zeros
-            cur_row0 = pg_ok ? pg * a.page_size : a.pool_pages * a.page_size - j0 % a.page_size;
+            cur_row0 = pg_ok ? pg * a.page_size : a.pool_pages * a.page_size - cur_off;
+            new_page = false;
           }
-          row = cur_row0 + j0 % a.page_size;
+          row = cur_row0 + cur_off;
+          cur_off += KB;
+          if (cur_off == a.page_size) {  // pages hold a multiple of KB keys
+            cur_off = 0;
+            ++cur_idx;
+            new_page = true;
+          }
         }
         mbar_arrive_expect_tx(&full[st], bytes);
         for (int hh = 0; hh < nheads; ++hh)
