@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/bifocal.h"
@@ -39,6 +40,12 @@ struct Rope {
 
 // omega_k = theta^(-2k/D) in fp64 on the host; long-range forms for factor G.
 Rope make_rope(double theta, int D, int G) {
+  // A decode loop asks for the same tables every step: keep the last set per thread (64 pow
+  // calls are a few microseconds of host time, as much as a short decode step takes on the GPU).
+  thread_local double last_theta = 0.0;
+  thread_local int last_D = 0, last_G = 0;
+  thread_local Rope last;
+  if (theta == last_theta && D == last_D && G == last_G) return last;
   Rope r;
   std::memset(&r, 0, sizeof(r));
   for (int k = 0; k < D / 2; ++k) {
@@ -47,6 +54,10 @@ Rope make_rope(double theta, int D, int G) {
     r.omega_long[k] = om / G;
     r.omega_corr[k] = om / G - om;
   }
+  last = r;
+  last_theta = theta;
+  last_D = D;
+  last_G = G;
   return r;
 }
 
@@ -71,9 +82,12 @@ float scale_log2(const bf_params_t* p) {
 }
 
 int sm_count() {
+  static std::atomic<int> cached[64];  // per device ordinal, 0 = not asked yet
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64 && (n = cached[dev].load(std::memory_order_relaxed)) > 0) return n;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -617,10 +631,28 @@ struct DecodeLayout {
 template <int D, bool TEST>
 cudaError_t launch_partial_t(dim3 grid, cudaStream_t st, const bf::DecodeArgs& da) {
   constexpr int smem = bf::decode_smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(bf::decode_partial_kernel<D, TEST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       smem);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(bf::decode_partial_kernel<D, TEST>, grid, dim3(bf::decode_threads<D>()), smem, st, da);
+  // The shared-memory limit is an attribute of the kernel in the current context: set it once
+  // per device rather than on every step, and again if a launch is refused (a context made anew
+  // after a device reset starts without it).
+  static std::atomic<bool> set_on[64];
+  auto set_attr = [&]() {
+    return cudaFuncSetAttribute(bf::decode_partial_kernel<D, TEST>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  };
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const bool known = dev >= 0 && dev < 64 && set_on[dev].load(std::memory_order_relaxed);
+  if (!known) {
+    const cudaError_t e = set_attr();
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) set_on[dev].store(true, std::memory_order_relaxed);
+  }
+  cudaError_t e = launch_pdl(bf::decode_partial_kernel<D, TEST>, grid, dim3(bf::decode_threads<D>()), smem, st, da);
+  if (e != cudaSuccess && known) {
+    (void)cudaGetLastError();
+    if (set_attr() == cudaSuccess)
+      e = launch_pdl(bf::decode_partial_kernel<D, TEST>, grid, dim3(bf::decode_threads<D>()), smem, st, da);
+  }
+  return e;
 }
 
 cudaError_t launch_partial(int D, dim3 grid, cudaStream_t st, const bf::DecodeArgs& da) {
