@@ -215,8 +215,10 @@ BF_API bf_status_t bifocal_prefill_chunk(const void* q, const void* k, const voi
  * chunk call; a sequence whose G is 1 or whose w0 >= its length runs the two-branch kernel (as with
  * BF_FLAG_FORCE_BIFOCAL, identical result). Pool rows past a sequence's end are never scored:
  * their key rows are zeroed in shared memory and their value rows too, whatever the pool holds.
- * block_table entries are trusted: every page a sequence's first P0_b + C_b positions use must be
- * a page of the pool.
+ * Every page a sequence's first P0_b + C_b positions use must be a page of the pool. The kernels
+ * check each entry they read: one outside [0, pool_pages) is reported as BF_ERR_INDEX by
+ * bifocal_last_device_error, its pool rows are not written and its key/value tiles read as zeros
+ * (the results of that sequence are then wrong, and nothing outside the pool is touched).
  * Errors: as bifocal_prefill_chunk; BF_ERR_INVALID also for batch < 1, a bad page_size, P0_b < 0,
  * C_b < 1, P0_b + C_b > max_pages * page_size or NULL arrays; BF_ERR_UNSUPPORTED for batch > 64,
  * head_dim != 128 or an odd GQA group. */
@@ -263,8 +265,11 @@ BF_API bf_status_t bifocal_decode(const void* q, const void* k_new, const void* 
  *   workspace / ws_bytes: >= bifocal_decode_paged_workspace_size(batch, max_len, p), 256-byte aligned.
  * Pages past a sequence's length are never read except the tail of its last 16-key stage, whose
  * keys are masked and whose values are zeroed in shared memory before use (an uninitialised
- * slot cannot turn the result into NaN). block_table entries and seq_lens are trusted: each
- * used entry must name a page of the pool.
+ * slot cannot turn the result into NaN). Each used block_table entry must name a page of the pool
+ * and each length lie in [1, max_len]. The kernels check both on the device: a length out of range
+ * appends nothing and gives NaN as that sequence's output; a table entry outside [0, pool_pages)
+ * is not written and its keys read as zeros; either is reported as BF_ERR_INDEX by
+ * bifocal_last_device_error, and nothing outside the pool, the table or the workspace is touched.
  * Errors: as bifocal_decode; BF_ERR_INVALID also for batch, pool_pages, max_pages or max_len < 1, a
  * page_size that is not a positive multiple of 16, max_pages * page_size < max_len or a NULL
  * table; BF_ERR_UNSUPPORTED for BF_FLAG_WINDOW. */
