@@ -34,3 +34,17 @@ def test_peaks_fall_back_when_the_measured_file_is_absent(monkeypatch):
     monkeypatch.setattr(bench, "ROOT", "/nonexistent")
     peaks, kind = bench.load_peaks()
     assert kind == "fallback" and peaks["bf16_tflops"] > 0 and peaks["hbm_gbs"] > 0
+
+
+def test_traffic_record_is_keyed_to_every_kernel_source():
+    # the record follows every source the prefill attention kernel compiles from
+    t = bench.TRAFFIC["prefill_attention"]
+    assert set(t["sources"]) >= {"common.cuh", "prefill_tc.cuh", "prefill_tc2.cuh", "rope_loads.cuh"}
+
+
+def test_roof_entry_reports_what_it_timed():
+    r = bench.roof("tensor", 826.1, 1652.2, "TFLOP/s", "chunked prefill", "whole call", "measured")
+    assert r["frac"] == 0.5 and r["bound"] == "tensor" and r["traffic"] is None
+    assert r["peak_kind"] == "measured bf16 dense burst" and r["scope"] == "whole call"
+    h = bench.roof("hbm", 3274.1, 6548.2, "GB/s", "paged decode", "whole step", "fallback", extra=1)
+    assert h["frac"] == 0.5 and h["peak_kind"] == "fallback HBM copy" and h["extra"] == 1
