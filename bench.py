@@ -165,6 +165,30 @@ class Clocks:
 
 
 # ------------------------------------------------------------------ timing helpers
+class nvtx_range:
+    """An NVTX range around one phase of the run (visible in a profiler's timeline); a no-op where
+    NVTX is unavailable. Host-side markers only: nothing is added on the device."""
+
+    def __init__(self, torch, name):
+        self.torch, self.name, self.on = torch, name, False
+
+    def __enter__(self):
+        try:
+            self.torch.cuda.nvtx.range_push(self.name)
+            self.on = True
+        except Exception:
+            self.on = False
+        return self
+
+    def __exit__(self, *exc):
+        if self.on:
+            try:
+                self.torch.cuda.nvtx.range_pop()
+            except Exception:
+                pass
+        return False
+
+
 def time_loop(fn, steps, warmup, dist, torch):
     """Device time of `steps` calls of fn (CUDA events on the current stream), max over ranks."""
     for _ in range(warmup):
@@ -343,13 +367,14 @@ def run_ours(args):
     clocks = Clocks(dist.local)
     clocks.start()
     time.sleep(0.3)
-    for i in range(args.steps):
-        ev[i][0].record()
-        step_rope()
-        ev[i][1].record()
-        step_attn()
-        ev[i][2].record()
-        launches += 2
+    with nvtx_range(torch, "headline: 128K prefill steps"):
+        for i in range(args.steps):
+            ev[i][0].record()
+            step_rope()
+            ev[i][1].record()
+            step_attn()
+            ev[i][2].record()
+            launches += 2
     torch.cuda.synchronize()
     clk = clocks.stop()
     dist.barrier()
@@ -505,17 +530,20 @@ def run_ours(args):
     if not args.no_decode:
         del ws
         torch.cuda.empty_cache()
-        decode = run_decode(args, torch, bfl, si, dev, peaks, peak_kind)
+        with nvtx_range(torch, "decode sessions"):
+            decode = run_decode(args, torch, bfl, si, dev, peaks, peak_kind)
 
     paged = None
     if not args.no_paged:
         torch.cuda.empty_cache()
-        paged = run_paged(args, torch, bfl, si, dev, peaks, peak_kind)
+        with nvtx_range(torch, "batched paged decode"):
+            paged = run_paged(args, torch, bfl, si, dev, peaks, peak_kind)
 
     chunk_paged = None
     if not args.no_chunk_paged:
         torch.cuda.empty_cache()
-        chunk_paged = run_chunk_paged(args, torch, bfl, si, dev, peak_t, peak_kind, dist)
+        with nvtx_range(torch, "batched paged chunked prefill"):
+            chunk_paged = run_chunk_paged(args, torch, bfl, si, dev, peak_t, peak_kind, dist)
 
     # ---- CPU baseline: the oracle on a bounded sample, rank 0, N = 1 only
     cpu = None

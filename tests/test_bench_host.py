@@ -48,3 +48,16 @@ def test_roof_entry_reports_what_it_timed():
     assert r["peak_kind"] == "measured bf16 dense burst" and r["scope"] == "whole call"
     h = bench.roof("hbm", 3274.1, 6548.2, "GB/s", "paged decode", "whole step", "fallback", extra=1)
     assert h["frac"] == 0.5 and h["peak_kind"] == "fallback HBM copy" and h["extra"] == 1
+
+
+def test_nvtx_range_is_a_no_op_without_nvtx():
+    import types
+    import torch
+    with bench.nvtx_range(torch, "phase"):  # real NVTX (a host-side marker) where torch has it
+        pass
+
+    class NoNvtx:
+        cuda = types.SimpleNamespace()  # no .nvtx attribute
+
+    with bench.nvtx_range(NoNvtx, "phase") as r:
+        assert r.on is False
