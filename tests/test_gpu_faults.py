@@ -3,14 +3,16 @@
 Two kinds of device-side event set the library's status word instead of trapping:
 
 - a bounded wait that expires. A test-only control makes the producer of one CTA skip a
-  whole fill (no expect_tx, no copy), so the wait for that fill can only run out; with the
-  wait limit shortened to 50 ms the call returns after about that long, every role of the
-  CTA leaves through its normal teardown (the producer first waits for each copy it did
-  issue, the MMA issuer for its MMAs, tensor memory is freed), and bifocal_last_device_error
-  reports BF_ERR_TIMEOUT with the site of the wait that gave up;
+  whole fill of the prefill kernel (no expect_tx, no copy), or stop issuing the decode kernel's
+  stages from a given one on (in a test-only instantiation of that kernel), so the wait for it
+  can only run out; with the wait limit shortened to 50 ms the call returns after about that
+  long, every role of the CTA leaves through its normal teardown (a producer that saw the expiry
+  first waits for each copy it did issue, the MMA issuer for its MMAs, tensor memory is freed),
+  and bifocal_last_device_error reports BF_ERR_TIMEOUT with the site of the wait that gave up;
 - an fp16 QK^T operand out of range: q scaled by 1e5 makes the rotated queries exceed 65520,
   which fp16 would round to inf; the RoPE pass (prefill) and the query rotation (decode)
-  report BF_ERR_RANGE.
+  report BF_ERR_RANGE, and a cached key of +-1e6 is caught by the decode kernel's check of its
+  final running max and sum.
 
 After each event the next normal call on the same device returns BF_OK and matches the oracle.
 """
