@@ -845,7 +845,7 @@ void* noalloc_scratch_ptr() {
 }  // namespace
 
 // ------------------------------------------------------------------ batched decode over a paged cache
-// Partial rows per sequence: two per split, splits <= min(kMaxSplits, ceil(max_len / KB)).
+// Partial rows per sequence: one per split, splits <= min(kMaxSplits, ceil(max_len / KB)).
 int paged_parts_stride(int max_len) { return std::min(kMaxSplits, (max_len + bf::dec::KB - 1) / bf::dec::KB); }
 
 size_t paged_workspace(int batch, int max_len, const bf_params_t* p) {

@@ -14,8 +14,8 @@
 // Work split: CTA = (key range, up to 4 kv heads). A TMA warp streams 16-key stages
 // (K and V, every head, both 64-element halves of D) through a 5-deep mbarrier ring, two
 // table warps build each stage's correction cos/sin table; two consumer warps per kv head each take
-// one 8-key n-tile of every stage, keeping their own online softmax (each warp is a split
-// of its own for the combine). QK^T of the
+// one 8-key n-tile of every stage, keeping their own online softmax, and merge the two states in
+// shared memory at the end, so each key range leaves one partial per query head. QK^T of the
 // g = hq/hkv query rows runs on mma.sync m16n8k16 (rows in M); PV runs transposed,
 // O^T = V^T P^T on m16n8k8, so the query rows sit in N and the accumulator is D x 8.
 // QK^T operands are fp16 (rotated query, corrected or converted cached key), PV is bf16.
@@ -35,8 +35,8 @@ struct DecodeArgs {
   CUtensorMap kmap;  // cache K viewed as (d_lo 64, d_hi D/64, head hkv, key cap), box (64,1,1,KB)
   CUtensorMap vmap;
   const __nv_bfloat16* q;  // [hq, D] raw
-  float* part_o;           // [2 * n_split, hq, D] unnormalised
-  float* part_ml;          // [2 * n_split, hq, 2]: running max (log2 domain), sum
+  float* part_o;           // [n_split, hq, D] unnormalised (batched: parts_stride rows per sequence)
+  float* part_ml;          // [n_split, hq, 2]: running max (log2 domain), sum
   int L, hq, hkv, w0, G, mode, bifocal;
   int key0;  // first key read: 0, or L - w0 for a sliding window
   int split_len, n_split;
