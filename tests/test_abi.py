@@ -53,11 +53,23 @@ def test_factor_matches_golden_table(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, 8):
+    for code in range(0, 9):
         assert isinstance(lib.bifocal_status_string(code), bytes)
     assert b"invalid" in lib.bifocal_status_string(1)
     assert b"workspace" in lib.bifocal_status_string(5)
+    assert b"fp16" in lib.bifocal_status_string(7)
+    assert b"block-table" in lib.bifocal_status_string(8)
+    assert b"unknown" in lib.bifocal_status_string(9)
     assert b"sm_100a" in lib.bifocal_build_info()
+
+
+def test_status_codes_agree_with_the_header():
+    import re
+    hdr = open(os.path.join(ROOT, "include", "bifocal.h")).read()
+    codes = dict((m.group(1), int(m.group(2))) for m in re.finditer(r"\b(BF_ERR_[A-Z_]+) = (\d+)", hdr))
+    assert codes["BF_ERR_TIMEOUT"] == bfl.STATUS_TIMEOUT
+    assert codes["BF_ERR_RANGE"] == bfl.STATUS_RANGE
+    assert codes["BF_ERR_INDEX"] == bfl.STATUS_INDEX
 
 
 def params(**kw):
